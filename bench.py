@@ -1,0 +1,389 @@
+"""Benchmark of the MapFlow hot path on B200.
+
+One step = one pass of the whole path over one sender layer and one receiver
+layer of the workload: block statistics (lse + block masses), selection and
+extraction of the kept blocks, and the fused map-mix x V.  Inputs are seeded
+and synthetic (shapes of the 32K-token workload by default) and already
+resident in HBM when the timed region starts; the kept map (tens of GB) is far
+larger than L2, so no separate L2 flush is done.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun), every rank runs an independent replica of the layer
+(the path has no exchange step): weak scaling, time = max over ranks.
+`--impl reference` times the CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from cross_model_attention_block_b200 import synth  # noqa: E402
+
+METRIC = ("mapped-AV GB/s & % HBM roofline; compress tokens/s & % tensor peak; "
+          "layer-prefill ms")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ reference arm
+
+def bench_reference(args, wl):
+    """Time the CPU oracle on bounded samples of the workload (rank 0)."""
+    from oracle import mapflow_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = len(os.sched_getaffinity(0))
+    x = synth.single_layer(wl)
+    L = wl.lengths[0]
+    B = wl.B
+    nqb = (L + B - 1) // B
+    per_step = 2
+    picks = [int((k + 0.5) * nqb / (per_step * (args.steps + args.warmup)))
+             for k in range(per_step * (args.steps + args.warmup))]
+    W = orc._f64(x.W)
+
+    def one(qb):
+        i1 = min(L, (qb + 1) * B)
+        Qs, Ks, Vs = orc._f64(x.Q[:i1]), orc._f64(x.K[:i1]), orc._f64(x.V[:i1])
+        r = orc.run_sequence(Qs, Ks, Vs, W, wl.Hkv, B, wl.tau, wl.band_bias, wl.band_width,
+                             qbs=[qb])
+        return r[qb]["O"].shape[0]
+
+    it = iter(picks)
+    for _ in range(args.warmup):
+        for _ in range(per_step):
+            one(next(it))
+    t0 = time.perf_counter()
+    rows = 0
+    for _ in range(args.steps):
+        for _ in range(per_step):
+            rows += one(next(it))
+    dt = time.perf_counter() - t0
+    value = rows / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": L, "Hs": wl.Hs, "Hr": wl.Hr,
+                   "Hkv": wl.Hkv, "d": wl.d, "B": wl.B, "tau": wl.tau},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} query blocks per step spread evenly over "
+                                   f"the {nqb} query blocks (causal cost averages out); "
+                                   f"full path per block"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_sample(wl, x, budget_s=20.0):
+    """The oracle on evenly spread query blocks until about budget_s of CPU work."""
+    from oracle import mapflow_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = len(os.sched_getaffinity(0))
+    L, B = wl.lengths[0], wl.B
+    nqb = (L + B - 1) // B
+    order = [int((k + 0.5) * nqb / 8) for k in range(8)]
+    W = orc._f64(x.W)
+    rows, done = 0, []
+    t0 = time.perf_counter()
+    for qb in order:
+        i1 = min(L, (qb + 1) * B)
+        r = orc.run_sequence(orc._f64(x.Q[:i1]), orc._f64(x.K[:i1]), orc._f64(x.V[:i1]), W,
+                             wl.Hkv, B, wl.tau, wl.band_bias, wl.band_width, qbs=[qb])
+        rows += r[qb]["O"].shape[0]
+        done.append(qb)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"query blocks {done} of {nqb} (rows {rows} of {L}), whole path "
+                      f"per block, {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------- our arm
+
+def algorithmic(wl, nnz):
+    """Per-launch algorithmic bytes / flops of the three kernels."""
+    L = wl.ntok
+    pairs = sum(l * (l + 1) // 2 for l in wl.lengths)
+    el = 2 if wl.dtype == "bf16" else 4
+    nqb = sum((l + wl.B - 1) // wl.B for l in wl.lengths)
+    map_bytes = nnz * wl.Hs * wl.B * wl.B * el
+    av_bytes = (map_bytes + L * wl.Hkv * wl.d * el + L * wl.Hr * wl.d * el
+                + wl.Hr * wl.Hs * el + 4 * nnz + 8 * (nqb + 1))
+    stats_flops = 2.0 * wl.d * pairs * wl.Hs          # one QK^T over the causal triangle
+    extract_bytes = map_bytes
+    av_flops = 2.0 * nnz * wl.B * wl.B * (wl.Hs * wl.Hr + wl.d * wl.Hr)
+    return dict(av_bytes=av_bytes, stats_flops=stats_flops, extract_bytes=extract_bytes,
+                av_flops=av_flops, map_bytes=map_bytes)
+
+
+def bench_ours(args, wl, rank, world, local_rank):
+    from cross_model_attention_block_b200 import mapflow as mfb
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    x = synth.single_layer(wl)
+    ctx = mfb.Context.make(wl.lengths, wl.Hs, wl.d, wl.B, wl.band_bias, wl.band_width,
+                           wl.torch_dtype, device=dev)
+    Q, K, V, W = (t.to(dev) for t in (x.Q, x.K, x.V, x.W))
+    nqb, nblocks = ctx.layout_sizes()
+    lse = torch.empty((wl.Hs, wl.ntok), dtype=torch.float32, device=dev)
+    mass = torch.empty((nblocks,), dtype=torch.float32, device=dev)
+    cache = mfb.Cache(ctx, device=dev)
+    O = torch.empty((wl.ntok, wl.Hr, wl.d), dtype=wl.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(marks=None):
+        if marks is not None:
+            marks[0].record(stream)
+        mfb.block_stats(ctx, Q, K, lse=lse, mass=mass)
+        if marks is not None:
+            marks[1].record(stream)
+        mfb.select_extract(ctx, Q, K, lse, mass, wl.tau, cache=cache)
+        if marks is not None:
+            marks[2].record(stream)
+        mfb.mapped_av(cache, wl.Hr, W, V, wl.Hkv, O=O)
+        if marks is not None:
+            marks[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    mfb.sync_status()
+    nnz = cache.nnz
+    alg = algorithmic(wl, nnz)
+
+    marks = [[ev() for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    t_start, t_end = ev(), ev()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(marks[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t_start.elapsed_time(t_end)
+    stage = np.array([[m[i].elapsed_time(m[i + 1]) for i in range(3)] for m in marks])
+    stage_ms = stage.mean(axis=0)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    mfb.sync_status()
+
+    # end to end through the C ABI: host inputs in, host output back
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    hQ, hK, hV, hW = pin(x.Q), pin(x.K), pin(x.V), pin(x.W)
+    hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    dQ, dK, dV, dW = (torch.empty_like(t, device=dev) for t in (hQ, hK, hV, hW))
+
+    def e2e_step():
+        dQ.copy_(hQ, non_blocking=True)
+        dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        dW.copy_(hW, non_blocking=True)
+        mfb.block_stats(ctx, dQ, dK, lse=lse, mass=mass)
+        mfb.select_extract(ctx, dQ, dK, lse, mass, wl.tau, cache=cache)
+        mfb.mapped_av(cache, wl.Hr, dW, dV, wl.Hkv, O=O)
+        hO.copy_(O, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    mfb.sync_status()
+    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hW))
+    d2h = hO.numel() * hO.element_size()
+
+    if rank != 0:
+        return
+    peaks, src = load_peaks()
+    ms_step = ms / args.steps
+    tokens = wl.ntok * world
+    t_stats, t_sel, t_av = stage_ms
+    av_gbs = alg["av_bytes"] / (t_av * 1e-3) / 1e9
+    stats_tf = alg["stats_flops"] / (t_stats * 1e-3) / 1e12
+    ext_gbs = alg["extract_bytes"] / (t_sel * 1e-3) / 1e9
+    hbm = peaks["hbm_gbs"]
+    tens = peaks["bf16_tflops"]
+    kernels = {
+        "mapped_av": {"bound": "hbm", "achieved": av_gbs, "peak": hbm, "unit": "GB/s",
+                      "frac": av_gbs / hbm, "ms": t_av,
+                      "algorithmic_bytes": alg["av_bytes"]},
+        "block_stats": {"bound": "tensor", "achieved": stats_tf, "peak": tens,
+                        "unit": "TFLOP/s", "frac": stats_tf / tens, "ms": t_stats,
+                        "algorithmic_flops": alg["stats_flops"]},
+        "select_extract": {"bound": "hbm", "achieved": ext_gbs, "peak": hbm, "unit": "GB/s",
+                           "frac": ext_gbs / hbm, "ms": t_sel,
+                           "algorithmic_bytes": alg["extract_bytes"]},
+    }
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    roof = {k: v for k, v in kernels[dom].items() if k in ("bound", "achieved", "peak", "unit",
+                                                            "frac")}
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{src} (MEASURED_PEAKS.json)" if src == "measured" else src
+    roof["traffic"] = None
+    line = {
+        "metric": METRIC, "value": tokens / (ms_step * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.ntok, "Hs": wl.Hs, "Hr": wl.Hr,
+                   "Hkv": wl.Hkv, "d": wl.d, "B": wl.B, "tau": wl.tau,
+                   "kept_blocks": nnz, "causal_blocks": nblocks,
+                   "map_gb": alg["map_bytes"] / 1e9,
+                   "l2": "inputs larger than L2 (kept map >> 126 MB); no flush",
+                   "parallelism": f"replicas{world}"},
+        "mapped_av_gbs": av_gbs, "mapped_av_hbm_frac": av_gbs / hbm,
+        "compress_tokens_per_s": wl.ntok / ((t_stats + t_sel) * 1e-3),
+        "stats_tensor_frac": stats_tf / tens,
+        "layer_prefill_ms": t_av,
+        "stage_ms": {"block_stats": t_stats, "select_extract": t_sel, "mapped_av": t_av},
+        "roofline": roof, "kernels": kernels,
+        "clocks": clk,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * LAUNCHES_PER_STEP,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sample(wl, x)
+    print(json.dumps(line), flush=True)
+
+
+# kernels of ours launched per step: stats (meta, stats, mass reduce), select and
+# extract (meta, qb map, select, scan, fill, extract), mapped AV (1)
+LAUNCHES_PER_STEP = 10
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="large_bf16_n32768")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = synth.workloads()[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            bench_reference(args, wl)
+        return 0
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        bench_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,265 @@
+// Host side of libmapflow: argument checks, workspace layout, dispatch to the
+// kernels, the device status word and the host prefix-hash index.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "mf_internal.h"
+
+namespace mf {
+
+__device__ unsigned g_status_word;
+
+namespace {
+thread_local std::string t_last_error;
+std::mutex g_status_mu;
+unsigned* g_status_ptr[64] = {nullptr};
+
+mf_status fail(mf_status st, const std::string& msg) {
+  t_last_error = msg;
+  return st;
+}
+
+mf_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(MF_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+}  // namespace
+
+unsigned* status_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+// ------------------------------------------------------------ validation
+
+static mf_status sizes_of(int32_t nseq, const int32_t* cu, int32_t B, Sizes* out) {
+  if (nseq < 1 || cu == nullptr) return fail(MF_ERR_INVALID_ARG, "nseq < 1 or cu_seqlens_host is NULL");
+  if (B != 64 && B != 128) return fail(MF_ERR_UNSUPPORTED, "block size B must be 64 or 128");
+  if (cu[0] != 0) return fail(MF_ERR_INVALID_ARG, "cu_seqlens_host[0] must be 0");
+  Sizes s;
+  for (int i = 0; i < nseq; ++i) {
+    int64_t L = int64_t(cu[i + 1]) - cu[i];
+    if (L < 0) return fail(MF_ERR_INVALID_ARG, "cu_seqlens_host must be non-decreasing");
+    if (L > int64_t(512) * B)
+      return fail(MF_ERR_UNSUPPORTED, "sequence longer than 512 blocks");
+    int64_t n = (L + B - 1) / B;
+    s.nqb += n;
+    s.nblocks += n * (n + 1) / 2;
+    s.ntiles += (L + 127) / 128;
+    if (L > s.max_len) s.max_len = int32_t(L);
+  }
+  s.ntok = cu[nseq];
+  *out = s;
+  return MF_OK;
+}
+
+static mf_status check_desc(const mf_attn_desc* d, Sizes* sz) {
+  if (!d) return fail(MF_ERR_INVALID_ARG, "desc is NULL");
+  if (!d->cu_seqlens) return fail(MF_ERR_INVALID_ARG, "cu_seqlens (device) is NULL");
+  mf_status st = sizes_of(d->nseq, d->cu_seqlens_host, d->B, sz);
+  if (st != MF_OK) return st;
+  if (d->Hs < 1 || d->Hs > 64) return fail(MF_ERR_UNSUPPORTED, "Hs must be in [1, 64]");
+  if (d->d != 64 && d->d != 128) return fail(MF_ERR_UNSUPPORTED, "head dim d must be 64 or 128");
+  if (d->dt != MF_BF16 && d->dt != MF_F32) return fail(MF_ERR_INVALID_ARG, "unknown dtype");
+  if (d->band_width < 0) return fail(MF_ERR_INVALID_ARG, "band_width < 0");
+  if (!std::isfinite(d->band_bias)) return fail(MF_ERR_INVALID_ARG, "band_bias not finite");
+  return MF_OK;
+}
+
+static size_t meta_bytes(Carve& c, int nseq, Meta* m) {
+  Meta mm;
+  mm.cu_qb = c.take<int32_t>(nseq + 1);
+  mm.cu_blk = c.take<int64_t>(nseq + 1);
+  mm.cu_tile = c.take<int32_t>(nseq + 1);
+  if (m) *m = mm;
+  return c.used;
+}
+
+static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+// ------------------------------------------------------------- stats
+
+static size_t stats_ws(const mf_attn_desc& d, const Sizes& sz, void* base, Meta* m,
+                       float** part) {
+  Carve c(base);
+  meta_bytes(c, d.nseq, m);
+  float* p = c.take<float>(size_t(d.Hs) * size_t(sz.nblocks));
+  if (part) *part = p;
+  return c.used + 256;
+}
+
+static size_t select_ws(const mf_attn_desc& d, const Sizes& sz, void* base, Meta* m,
+                        int32_t** counts, uint8_t** keep, int32_t** slot) {
+  Carve c(base);
+  meta_bytes(c, d.nseq, m);
+  int32_t* a = c.take<int32_t>(size_t(sz.nqb) + 1);
+  uint8_t* b = c.take<uint8_t>(size_t(sz.nblocks) + 1);
+  int32_t* s = c.take<int32_t>(size_t(sz.nblocks) + 1);
+  if (counts) *counts = a;
+  if (keep) *keep = b;
+  if (slot) *slot = s;
+  return c.used + 256;
+}
+
+}  // namespace mf
+
+using namespace mf;
+
+extern "C" {
+
+const char* mf_version(void) { return "mapflow-b200 0.1 (sm_100a)"; }
+
+const char* mf_last_error(void) { return t_last_error.c_str(); }
+
+mf_status mf_layout_sizes(int32_t nseq, const int32_t* cu_seqlens_host, int32_t B,
+                          int64_t* nqb_total, int64_t* nblocks_total) {
+  Sizes sz;
+  mf_status st = sizes_of(nseq, cu_seqlens_host, B, &sz);
+  if (st != MF_OK) return st;
+  if (nqb_total) *nqb_total = sz.nqb;
+  if (nblocks_total) *nblocks_total = sz.nblocks;
+  return MF_OK;
+}
+
+size_t mf_block_stats_workspace(const mf_attn_desc* desc) {
+  Sizes sz;
+  if (check_desc(desc, &sz) != MF_OK) return 0;
+  return stats_ws(*desc, sz, nullptr, nullptr, nullptr);
+}
+
+mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K, float* lse,
+                         float* mass, void* ws, size_t ws_bytes, mf_stream_t stream) {
+  Sizes sz;
+  mf_status st = check_desc(desc, &sz);
+  if (st != MF_OK) return st;
+  if (!Q || !K || !lse || !mass) return fail(MF_ERR_INVALID_ARG, "Q, K, lse or mass is NULL");
+  const mf_attn_desc& d = *desc;
+  if (!ws || !aligned256(ws) || ws_bytes < stats_ws(d, sz, nullptr, nullptr, nullptr))
+    return fail(MF_ERR_WORKSPACE, "workspace missing, not 256-byte aligned or too small");
+  if (!status_word()) return fail(MF_ERR_CUDA, "no CUDA device");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Meta m;
+  float* part = nullptr;
+  stats_ws(d, sz, ws, &m, &part);
+  cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, m, s);
+  if (e != cudaSuccess) return cuda_fail(e, "meta");
+  if (sz.nqb == 0) return MF_OK;
+  e = launch_stats_simt(d, sz, m, Q, K, lse, part, s);
+  if (e != cudaSuccess) return cuda_fail(e, "block stats");
+  e = launch_mass_reduce(part, d.Hs, sz.nblocks, mass, s);
+  if (e != cudaSuccess) return cuda_fail(e, "mass reduce");
+  return MF_OK;
+}
+
+size_t mf_select_extract_workspace(const mf_attn_desc* desc) {
+  Sizes sz;
+  if (check_desc(desc, &sz) != MF_OK) return 0;
+  return select_ws(*desc, sz, nullptr, nullptr, nullptr, nullptr, nullptr);
+}
+
+static mf_status check_cache(const mf_csr_cache* c, const mf_attn_desc& d, const Sizes& sz) {
+  if (!c) return fail(MF_ERR_INVALID_ARG, "cache is NULL");
+  if (!c->row_ptr || !c->col_idx || !c->qb_seq || !c->qb_idx || !c->values)
+    return fail(MF_ERR_INVALID_ARG, "cache has a NULL array");
+  if (c->Hs != d.Hs || c->B != d.B || c->dt != d.dt)
+    return fail(MF_ERR_INVALID_ARG, "cache Hs/B/dtype differ from the descriptor");
+  if (c->nqb_total != sz.nqb)
+    return fail(MF_ERR_INVALID_ARG, "cache nqb_total differs from the context layout");
+  if (c->nnz_capacity < 0) return fail(MF_ERR_INVALID_ARG, "negative nnz_capacity");
+  return MF_OK;
+}
+
+mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void* K,
+                            const float* lse, const float* mass, double tau,
+                            mf_csr_cache* out, void* ws, size_t ws_bytes, mf_stream_t stream) {
+  Sizes sz;
+  mf_status st = check_desc(desc, &sz);
+  if (st != MF_OK) return st;
+  const mf_attn_desc& d = *desc;
+  if (!Q || !K || !lse || !mass) return fail(MF_ERR_INVALID_ARG, "Q, K, lse or mass is NULL");
+  if (!(tau > 0.0) || !std::isfinite(tau)) return fail(MF_ERR_INVALID_ARG, "tau must be > 0");
+  st = check_cache(out, d, sz);
+  if (st != MF_OK) return st;
+  if (!ws || !aligned256(ws) ||
+      ws_bytes < select_ws(d, sz, nullptr, nullptr, nullptr, nullptr, nullptr))
+    return fail(MF_ERR_WORKSPACE, "workspace missing, not 256-byte aligned or too small");
+  if (!status_word()) return fail(MF_ERR_CUDA, "no CUDA device");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Meta m;
+  int32_t* counts = nullptr;
+  uint8_t* keep = nullptr;
+  int32_t* slot = nullptr;
+  select_ws(d, sz, ws, &m, &counts, &keep, &slot);
+  cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, m, s);
+  if (e != cudaSuccess) return cuda_fail(e, "meta");
+  if (sz.nqb == 0) {
+    e = cudaMemsetAsync(out->row_ptr, 0, sizeof(int64_t), s);
+    return e == cudaSuccess ? MF_OK : cuda_fail(e, "row_ptr");
+  }
+  e = launch_select(d, sz, m, mass, tau, *out, counts, keep, slot, s);
+  if (e != cudaSuccess) return cuda_fail(e, "select");
+  e = launch_extract_simt(d, sz, Q, K, lse, *out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "extract");
+  return MF_OK;
+}
+
+mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int32_t Hr,
+                       const void* W, const mf_v_desc* v, void* O, mf_stream_t stream) {
+  Sizes sz;
+  mf_status st = check_desc(desc, &sz);
+  if (st != MF_OK) return st;
+  const mf_attn_desc& d = *desc;
+  st = check_cache(cache, d, sz);
+  if (st != MF_OK) return st;
+  if (!W || !v || !v->V || !O) return fail(MF_ERR_INVALID_ARG, "W, V or O is NULL");
+  if (v->d != d.d) return fail(MF_ERR_INVALID_ARG, "V head dim differs from the descriptor");
+  if (v->Hkv < 1 || Hr < 1 || Hr % v->Hkv != 0)
+    return fail(MF_ERR_INVALID_ARG, "Hr must be a positive multiple of Hkv");
+  if (int64_t(Hr) * d.d > 4096) return fail(MF_ERR_UNSUPPORTED, "Hr * d above 4096");
+  if (v->page_table) {
+    if (v->page_size < 16 || v->page_size % 16 != 0)
+      return fail(MF_ERR_INVALID_ARG, "page_size must be a positive multiple of 16");
+    if (int64_t(v->max_pages_per_seq) * v->page_size < sz.max_len)
+      return fail(MF_ERR_INVALID_ARG, "max_pages_per_seq * page_size below a sequence length");
+  }
+  if (!status_word()) return fail(MF_ERR_CUDA, "no CUDA device");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (sz.nqb == 0) return MF_OK;
+  cudaError_t e = launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, s);
+  if (e != cudaSuccess) return cuda_fail(e, "mapped av");
+  return MF_OK;
+}
+
+mf_status mf_sync_status(mf_stream_t stream) {
+  unsigned* p = status_word();
+  if (!p) return fail(MF_ERR_CUDA, "no CUDA device");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned v = 0;
+  e = cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (v != 0) {
+    unsigned zero = 0;
+    e = cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  }
+  if (v & kStatusTimeout) return fail(MF_ERR_TIMEOUT, "a device-side bounded wait gave up");
+  if (v & kStatusCapacity) return fail(MF_ERR_CAPACITY, "kept blocks exceed nnz_capacity");
+  return MF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,70 @@
+// Internal host-side interface between the translation units of libmapflow.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/mapflow.h"
+
+namespace mf {
+
+// Bits of the per-device status word.
+enum : unsigned { kStatusTimeout = 1u, kStatusCapacity = 2u };
+
+// Device address of the status word of the current device.
+unsigned* status_word();
+
+// Per-context block layout, device arrays computed from cu_seqlens.
+struct Meta {
+  int32_t* cu_qb;    // [nseq+1] prefix of ceil(L_s/B)
+  int64_t* cu_blk;   // [nseq+1] prefix of C_s
+  int32_t* cu_tile;  // [nseq+1] prefix of ceil(L_s/128)
+};
+
+// Host-side sizes of a context.
+struct Sizes {
+  int64_t ntok = 0;
+  int64_t nqb = 0;
+  int64_t nblocks = 0;
+  int64_t ntiles = 0;  // 128-row tiles
+  int32_t max_len = 0;
+};
+
+// Bump allocator over a caller workspace (256-byte aligned pieces).
+struct Carve {
+  char* base;
+  size_t used = 0;
+  explicit Carve(void* p) : base(static_cast<char*>(p)) {}
+  template <typename T>
+  T* take(size_t count) {
+    used = (used + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += count * sizeof(T);
+    return p;
+  }
+};
+
+// ---- launchers (return cudaGetLastError of the launch) ----
+cudaError_t launch_meta(int nseq, const int32_t* cu_seqlens, int B, const Meta& m,
+                        cudaStream_t st);
+
+cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
+                              const void* Q, const void* K, float* lse, float* part,
+                              cudaStream_t st);
+cudaError_t launch_mass_reduce(const float* part, int Hs, int64_t nblocks, float* mass,
+                               cudaStream_t st);
+
+cudaError_t launch_select(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
+                          const float* mass, double tau, const mf_csr_cache& c,
+                          int32_t* counts, uint8_t* keep, int32_t* slot, cudaStream_t st);
+
+cudaError_t launch_extract_simt(const mf_attn_desc& d, const Sizes& sz, const void* Q,
+                                const void* K, const float* lse, const mf_csr_cache& c,
+                                cudaStream_t st);
+
+cudaError_t launch_mapped_av_simt(const mf_csr_cache& c, const mf_attn_desc& d,
+                                  const Sizes& sz, int Hr, const void* W,
+                                  const mf_v_desc& v, void* O, cudaStream_t st);
+
+}  // namespace mf

@@ -1,0 +1,217 @@
+/*
+ * mapflow.h -- C ABI of libmapflow.so, the MapFlow hot path on B200 (sm_100a).
+ *
+ * MapFlow ("Accelerating Cross-Model LLM Inference via Attention Map Reuse",
+ * PKU-DAIR; 163.com article, section on the three system components) reuses a
+ * sender model's attention map in a receiver model.  The map is compressed to
+ * regular 2-D blocks kept by cumulative attention probability, in stages that
+ * never form the dense N x N matrix (block statistics, then extraction of the
+ * kept blocks).  A fused kernel reads the kept blocks, combines sender heads
+ * into receiver heads with a learned linear map W on chip, and multiplies the
+ * result into the receiver's own V.  A prefix-hash index lets a receiver find
+ * the cached state of a shared context.
+ *
+ * Conventions for every entry point:
+ *  - Plain pointers and sizes only.  "device" pointers are CUDA global memory
+ *    of the current device; "host" pointers are CPU memory.
+ *  - The caller owns every buffer.  The library never allocates device memory;
+ *    scratch space comes from a caller-provided workspace whose size the
+ *    matching *_workspace() query returns (bytes, 256-byte aligned start).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and is asynchronous.  Argument errors are found on the host
+ *    before anything is enqueued and return a status; nothing is enqueued
+ *    then.  Launch failures return MF_ERR_CUDA.  Conditions found on the
+ *    device (a bounded wait that gave up, a CSR capacity overflow) set a
+ *    per-device status word that mf_sync_status() reads and clears.
+ *  - The text of the last error of the calling thread: mf_last_error().
+ *
+ * Notation: ntok packed tokens over nseq sequences (cu_seqlens prefix sums);
+ * Hs sender heads; Hr receiver heads; Hkv receiver KV heads; d head dim;
+ * B block size.  Sequence s has L_s tokens, nqb_s = ceil(L_s / B) query
+ * blocks and C_s = nqb_s (nqb_s + 1) / 2 causal blocks; blocks are aligned to
+ * the start of each sequence and no token attends across sequences.
+ */
+#ifndef MAPFLOW_H
+#define MAPFLOW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mf_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  MF_OK = 0,
+  MF_ERR_INVALID_ARG = 1,  /* null pointer, inconsistent sizes */
+  MF_ERR_UNSUPPORTED = 2,  /* a shape this build has no kernel for */
+  MF_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
+  MF_ERR_CUDA = 4,         /* a CUDA runtime call or a launch failed */
+  MF_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up */
+  MF_ERR_NOT_FOUND = 6,    /* prefix index lookup found no match */
+  MF_ERR_CAPACITY = 7      /* kept blocks exceed the CSR capacity */
+} mf_status;
+
+typedef enum { MF_BF16 = 0, MF_F32 = 1 } mf_dtype;
+
+/* One sender layer's context.
+ * Logits (article: attention map of the sender, causal):
+ *   s_h[i,j] = q_i.k_j / sqrt(d) + band_bias * [0 <= i-j < band_width], j <= i.
+ * Q, K: device, [ntok][Hs][d] of dtype dt, row-major (token, head, dim).
+ * Supported: B in {64,128}, d in {64,128}, 1 <= Hs <= 64, L_s <= 512 * B.
+ * The bf16 tensor-core kernels need d = 128. */
+typedef struct {
+  int32_t nseq;
+  const int32_t* cu_seqlens;      /* device [nseq+1], cu_seqlens[0] = 0 */
+  const int32_t* cu_seqlens_host; /* host [nseq+1], the same values */
+  int32_t Hs, d, B;
+  float band_bias;
+  int32_t band_width;
+  mf_dtype dt;
+} mf_attn_desc;
+
+/* Block-sparse attention-map cache, CSR by query block (article: kept 2-D
+ * blocks, a variable number per layer and position).  All pointers are
+ * device memory owned by the caller; mf_select_extract fills them.
+ *  row_ptr [nqb_total+1] int64: kept blocks of global query block q are
+ *          entries row_ptr[q] .. row_ptr[q+1]-1.  Global query blocks are
+ *          numbered sequence by sequence.
+ *  col_idx [nnz_capacity] int32: key-block index within the sequence,
+ *          ascending within a row.
+ *  qb_seq, qb_idx [nqb_total] int32: sequence and in-sequence index of each
+ *          global query block.
+ *  values: kept probability blocks P_h[i,j] = exp(s_h[i,j] - lse_h[i]) for
+ *          j <= i (0 above the diagonal and beyond the sequence end), of
+ *          dtype dt, layout [nnz][B/16][B][Hs][16]: entry e, key group
+ *          jg = j/16, row i, head h, key j%16 -- except that the two 8-key
+ *          halves of the 16 keys are stored swapped when bit 2 of h is set
+ *          (stored position (j%16) ^ (8 * ((h>>2)&1))).
+ *  cu_seqlens, nseq: the context the cache was built from (device). */
+typedef struct {
+  int64_t nqb_total;
+  int64_t nnz_capacity;
+  int64_t* row_ptr;
+  int32_t* col_idx;
+  int32_t* qb_seq;
+  int32_t* qb_idx;
+  void* values;
+  int32_t Hs, B;
+  mf_dtype dt;
+  int32_t nseq;
+  const int32_t* cu_seqlens;
+} mf_csr_cache;
+
+/* Receiver V (article: the receiver keeps its own V; PagedAttention and
+ * varlen packing are supported).
+ *  page_table == NULL: V is [ntok][Hkv][d] (packed like Q).
+ *  otherwise V is a page pool [npages][page_size][Hkv][d] and
+ *  page_table[s * max_pages_per_seq + p] is the pool page holding tokens
+ *  p*page_size .. of sequence s.  page_size must be a multiple of 16. */
+typedef struct {
+  const void* V;
+  const int32_t* page_table;
+  int32_t page_size;
+  int32_t max_pages_per_seq;
+  int32_t Hkv, d;
+} mf_v_desc;
+
+/* Library version string. */
+const char* mf_version(void);
+
+/* Text of the last error returned to this thread ("" if none). */
+const char* mf_last_error(void);
+
+/* Sizes of the block layout for a context (host only).
+ * nqb_total = sum_s ceil(L_s/B); nblocks_total = sum_s C_s.  The mass array
+ * of mf_block_stats has nblocks_total entries; nblocks_total is also the
+ * CSR capacity that can never overflow. */
+mf_status mf_layout_sizes(int32_t nseq, const int32_t* cu_seqlens_host, int32_t B,
+                          int64_t* nqb_total, int64_t* nblocks_total);
+
+/* Stage 1, block statistics (article: block-level statistics first, with no
+ * dense N x N matrix).
+ *  lse  [Hs][ntok] float (device, out): natural-log log-sum-exp of each
+ *       causal row, lse_h[i] = log sum_{j<=i} exp(s_h[i,j]).
+ *  mass [nblocks_total] float (device, out): block (s, qb, kb), kb <= qb, at
+ *       index cu_blocks[s] + qb (qb+1)/2 + kb, where cu_blocks is the prefix
+ *       sum of C_s; mass = sum_h sum_{i in qb} sum_{j in kb, j<=i}
+ *       exp(s_h[i,j] - lse_h[i]).  Per-head partial sums are added in
+ *       float64 in head order, so results do not depend on scheduling.
+ *  ws: device workspace of at least mf_block_stats_workspace(desc) bytes. */
+size_t mf_block_stats_workspace(const mf_attn_desc* desc);
+mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
+                         float* lse, float* mass, void* ws, size_t ws_bytes,
+                         mf_stream_t stream);
+
+/* Stage 2, selection and extraction (article: keep the important blocks by
+ * cumulative attention probability; extract only the kept blocks).
+ * Per global query block: order key blocks by mass descending, ties to the
+ * lower index; take float64 prefix sums c_k in that order, T = c_last; keep
+ * the first k* = min{k : c_k >= tau * T} blocks (all blocks if tau >= 1);
+ * write them ascending into the CSR and write their probability blocks.
+ *  out: caller-filled descriptor (pointers, nqb_total, nnz_capacity, Hs, B,
+ *       dt, nseq, cu_seqlens); Hs/B/dt must match desc.
+ *  Overflowing nnz_capacity sets the device status (MF_ERR_CAPACITY via
+ *  mf_sync_status); entries past the capacity are dropped and the
+ *  results are incomplete. */
+size_t mf_select_extract_workspace(const mf_attn_desc* desc);
+mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void* K,
+                            const float* lse, const float* mass, double tau,
+                            mf_csr_cache* out, void* ws, size_t ws_bytes,
+                            mf_stream_t stream);
+
+/* Stage 3, fused map-mix x V (article: the fused kernel reads the sparse
+ * blocks, combines heads on chip and multiplies straight into the receiver's
+ * V, accumulating the output):
+ *   O_r[i,:] = sum_{kb kept for qb(i)} sum_{j in kb}
+ *              (sum_h W[r,h] P_h[i,j]) V_{g(r)}[j,:],  g(r) = floor(r*Hkv/Hr).
+ *  desc: the sender context (cu_seqlens, Hs, B, dt as in the cache).
+ *  W [Hr][Hs] of dtype dt (device); O [ntok][Hr][d] of dtype dt (device, out;
+ *  every row of every sequence is written).  No renormalisation of the kept
+ *  map.  Hr must be a multiple of Hkv. */
+mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc,
+                       int32_t Hr, const void* W, const mf_v_desc* v, void* O,
+                       mf_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the device status word of the
+ * current device: MF_OK, MF_ERR_TIMEOUT or MF_ERR_CAPACITY. */
+mf_status mf_sync_status(mf_stream_t stream);
+
+/* ---- host-side prefix index (article: states are indexed by a prefix hash
+ * that includes the preceding context; one sender state can serve several
+ * receivers).  The index stores cache descriptors, not copies: the caller
+ * keeps the buffers alive.  Not thread-safe per index object. */
+
+/* Chained 128-bit hash per block of B tokens: block k hashes the previous
+ * block's hash and its own tokens (two independent 64-bit FNV-1a chains).
+ * out [ceil(n/B)][2] (host).  A partial last block is hashed over the tokens
+ * it has. */
+mf_status mf_prefix_hash(const int32_t* tokens, int64_t n, int32_t B, uint64_t seed,
+                         uint64_t* out);
+
+mf_status mf_index_create(void** index);
+void mf_index_destroy(void* index);
+
+/* Registers every prefix 1..nblocks of a context (hashes [nblocks][2]) for
+ * sequence `seq` of `cache` at `sender_layer`.  A key already present is
+ * replaced (the newest insert wins). */
+mf_status mf_index_insert(void* index, const uint64_t* hashes, int64_t nblocks,
+                          int32_t sender_layer, int32_t seq, const mf_csr_cache* cache);
+
+/* Longest registered prefix of the query context (hashes [nblocks][2]) at
+ * `sender_layer`: fills *cache, *seq and *matched_blocks, or returns
+ * MF_ERR_NOT_FOUND (outputs untouched). */
+mf_status mf_index_lookup(void* index, const uint64_t* hashes, int64_t nblocks,
+                          int32_t sender_layer, mf_csr_cache* cache, int32_t* seq,
+                          int64_t* matched_blocks);
+
+/* Number of entries (prefix keys) held by the index. */
+int64_t mf_index_size(void* index);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAPFLOW_H */

@@ -132,7 +132,7 @@ def mixed_map(P: np.ndarray, kept: np.ndarray, W: np.ndarray, B: int) -> np.ndar
     for kb in kept:
         mask[kb * B:min(L1, (kb + 1) * B)] = True
     Pk = np.where(mask[None, None, :], P, 0.0)
-    return np.einsum("rh,hij->rij", W, Pk)
+    return np.tensordot(W, Pk, axes=(1, 0))      # sum over h
 
 
 def mapped_av(M: np.ndarray, V: np.ndarray, Hkv: int) -> np.ndarray:

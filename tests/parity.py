@@ -1,0 +1,162 @@
+"""Helpers that compare the CUDA path (through the C ABI) with the CPU oracle.
+
+Tolerances (from the stated acceptance rule of the hot path):
+* kept block sets bit-exact, except query blocks whose oracle cumulative mass
+  fraction at the cut lies within 1e-4 of tau, or whose only difference is a
+  swap of blocks with oracle masses closer than 1e-6 * T; these are counted;
+* O: max-abs error <= 2e-2 * max|O| for bf16, <= 1e-4 * max|O| for fp32;
+* lse, block masses and extracted probabilities: the float32 arithmetic of
+  the kernels on identical (rounded) inputs; bounds are stated per check.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from cross_model_attention_block_b200 import mapflow as mfb
+from oracle import mapflow_oracle as orc
+
+NEAR_TAU = 1e-4
+NEAR_SWAP = 1e-6
+
+
+def o_tol(dtype):
+    return 1e-4 if dtype == torch.float32 else 2e-2
+
+
+def run_gpu(ctx, Q, K, V, W, Hkv, tau, page_table=None, page_size=16, Vpool=None):
+    """The whole path through the C ABI; returns (lse, mass, cache, O)."""
+    lse, mass = mfb.block_stats(ctx, Q, K)
+    cache = mfb.select_extract(ctx, Q, K, lse, mass, tau)
+    if page_table is None:
+        O = mfb.mapped_av(cache, W.shape[0], W, V, Hkv)
+    else:
+        O = mfb.mapped_av(cache, W.shape[0], W, Vpool, Hkv, page_table=page_table,
+                          page_size=page_size)
+    mfb.sync_status()
+    return lse, mass, cache, O
+
+
+def kept_sets(cache):
+    rp = cache.row_ptr.cpu().numpy()
+    ci = cache.col_idx.cpu().numpy()
+    return rp, ci
+
+
+def check_selection(oracle_mass, gpu_kept, tau):
+    """0 if equal, 1 if the difference is exempt, raises otherwise."""
+    oracle_kept = orc.select_blocks(oracle_mass, tau)
+    if list(oracle_kept) == list(gpu_kept):
+        return 0
+    order, frac = orc.cumulative_fractions(oracle_mass)
+    k = len(oracle_kept)
+    near = [abs(frac[k - 1] - tau)]
+    if k >= 2:
+        near.append(abs(frac[k - 2] - tau))
+    if min(near) < NEAR_TAU:
+        return 1
+    T = oracle_mass.sum()
+    a, b = set(oracle_kept.tolist()), set(int(x) for x in gpu_kept)
+    if len(a) == len(b):
+        diff = sorted(a ^ b)
+        if max(oracle_mass[diff]) - min(oracle_mass[diff]) < NEAR_SWAP * T:
+            return 1
+    raise AssertionError(f"kept sets differ beyond the exemptions: oracle {sorted(a)} "
+                         f"gpu {sorted(b)}; cut fractions {near}")
+
+
+def f64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def block_index(cu_blk_s, qb, kb):
+    return cu_blk_s + qb * (qb + 1) // 2 + kb
+
+
+def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
+                         check_values=True, lse_atol=None):
+    """Compare the GPU result on selected (seq, qb) pairs with the oracle.
+
+    Qc, Kc, Vc, Wc are the CPU copies of the inputs (contiguous V).
+    Returns (n_checked, n_exempt, max_rel_err_O).
+    """
+    lse_g, mass_g, cache, O_g = gpu
+    B = ctx.B
+    cu = ctx.cu_seqlens_host
+    lens = np.diff(cu)
+    nqb = (lens + B - 1) // B
+    cu_qb = np.concatenate([[0], np.cumsum(nqb)])
+    cu_blk = np.concatenate([[0], np.cumsum(nqb * (nqb + 1) // 2)])
+    rp, ci = kept_sets(cache)
+    lse_g = lse_g.cpu().numpy()
+    mass_g = mass_g.cpu().numpy()
+    W = f64(Wc)
+    vals = cache.values_view() if check_values else None
+    n_ex = 0
+    worst = 0.0
+    tol = o_tol(dtype)
+    if lse_atol is None:
+        lse_atol = 2e-5 if dtype == torch.float32 else 1e-4
+    for s, qb in picks:
+        s0, L = int(cu[s]), int(lens[s])
+        i0, i1 = qb * B, min(L, (qb + 1) * B)
+        Qs = f64(Qc[s0:s0 + i1])
+        Ks = f64(Kc[s0:s0 + i1])
+        Vs = f64(Vc[s0:s0 + i1])
+        lse_o, P, mass_o = orc.query_block(Qs, Ks, qb, B, ctx.band_bias, ctx.band_width)
+        # lse
+        np.testing.assert_allclose(lse_g[:, s0 + i0:s0 + i1], lse_o, rtol=0, atol=lse_atol,
+                                   err_msg=f"lse seq {s} qb {qb}")
+        # block masses (float32 sums of float32 terms)
+        b0 = block_index(cu_blk[s], qb, 0)
+        T = mass_o.sum()
+        np.testing.assert_allclose(mass_g[b0:b0 + qb + 1], mass_o, rtol=0, atol=2e-5 * T,
+                                   err_msg=f"mass seq {s} qb {qb}")
+        # selection
+        g = int(cu_qb[s] + qb)
+        kept_g = ci[rp[g]:rp[g + 1]]
+        assert np.all(np.diff(kept_g) > 0), "kept blocks not ascending"
+        ex = check_selection(mass_o, kept_g, tau)
+        n_ex += ex
+        if ex:
+            continue
+        # extracted probability blocks
+        if check_values:
+            for e, kb in zip(range(rp[g], rp[g + 1]), kept_g):
+                blk = f64(vals[e])                       # [B/16, B, Hs, 16] stored order
+                ref = np.zeros((P.shape[0], B, B))
+                hi = min(P.shape[2], (kb + 1) * B)
+                ref[:, : i1 - i0, : hi - kb * B] = P[:, :, kb * B:hi]
+                got = unswizzle_block(blk, ctx.Hs, B)    # [Hs, B, B]
+                if dtype == torch.float32:
+                    np.testing.assert_allclose(got, ref, rtol=2e-5, atol=1e-7)
+                else:
+                    np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-6)
+        # output rows
+        M = orc.mixed_map(P, np.array(kept_g), W, B)
+        O_o = orc.mapped_av(M, Vs, Hkv)
+        O_gpu = f64(O_g[s0 + i0:s0 + i1])
+        scale = max(np.abs(O_o).max(), 1e-30)
+        err = np.abs(O_gpu - O_o).max() / scale
+        worst = max(worst, err)
+        assert err <= tol, f"O seq {s} qb {qb}: rel err {err:.3e} > {tol}"
+    return len(picks), n_ex, worst
+
+
+def unswizzle_block(blk, Hs, B):
+    """Stored [B/16, B, Hs, 16] (halves swapped for heads with bit 2 set) ->
+    logical [Hs, B rows, B keys]."""
+    out = np.empty((Hs, B, B))
+    for h in range(Hs):
+        sw = 8 if (h >> 2) & 1 else 0
+        idx = np.arange(16) ^ sw              # logical key -> stored slot
+        grp = blk[:, :, h, :][:, :, idx]      # [B/16, B, 16] logical keys
+        out[h] = np.transpose(grp, (1, 0, 2)).reshape(B, B)
+    return out
+
+
+def all_picks(ctx):
+    cu = ctx.cu_seqlens_host
+    B = ctx.B
+    return [(s, qb) for s in range(len(cu) - 1)
+            for qb in range((int(cu[s + 1] - cu[s]) + B - 1) // B)]

@@ -1,0 +1,158 @@
+"""Host-side checks of the C ABI: exports, layout sizes, argument validation,
+and the prefix-hash index (no GPU needed; nothing here launches a kernel)."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+from cross_model_attention_block_b200 import mapflow as mfb
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "mapflow.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mf_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert "mf_mapped_av" in names and len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(mfb.EXPORTED) <= set(names)
+    assert lib.mf_version().decode().startswith("mapflow")
+
+
+def _sizes_py(lengths, B):
+    nqb = sum((L + B - 1) // B for L in lengths)
+    nbl = sum(((L + B - 1) // B) * ((L + B - 1) // B + 1) // 2 for L in lengths)
+    return nqb, nbl
+
+
+@pytest.mark.parametrize("lengths,B", [([512], 64), ([8192], 64), ([32768], 128),
+                                       ([1, 63, 64, 65, 0, 1000], 64), ([130, 7], 128)])
+def test_layout_sizes(lib, lengths, B):
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    assert mfb.layout_sizes(cu, B) == _sizes_py(lengths, B)
+
+
+def test_layout_sizes_rejects_bad_input(lib):
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.layout_sizes(np.array([0, 100], np.int32), 32)
+    assert e.value.status == mfb.MF_ERR_UNSUPPORTED
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.layout_sizes(np.array([0, 100, 50], np.int32), 64)
+    assert e.value.status == mfb.MF_ERR_INVALID_ARG
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.layout_sizes(np.array([0, 512 * 64 + 1], np.int32), 64)
+    assert e.value.status == mfb.MF_ERR_UNSUPPORTED
+
+
+def _desc(Hs=4, d=64, B=64, cu=(0, 512), dt=mfb.MF_F32):
+    host = np.array(cu, dtype=np.int32)
+    dsc = mfb.AttnDesc(len(cu) - 1, 0x1000, host.ctypes.data, Hs, d, B, 0.0, 256, dt)
+    return dsc, host
+
+
+def test_argument_errors_return_before_any_launch(lib):
+    dsc, host = _desc()
+    P = C.c_void_p
+    # NULL descriptor
+    assert lib.mf_block_stats(None, P(16), P(16), P(16), P(16), P(256), 1 << 20, None) == \
+        mfb.MF_ERR_INVALID_ARG
+    # unsupported head dim / Hs
+    for bad in (dict(d=96), dict(Hs=65), dict(B=32)):
+        b, h = _desc(**bad)
+        st = lib.mf_block_stats(C.byref(b), P(16), P(16), P(16), P(16), P(256), 1 << 20, None)
+        assert st == mfb.MF_ERR_UNSUPPORTED, bad
+        assert lib.mf_last_error().decode()
+    # NULL inputs
+    assert lib.mf_block_stats(C.byref(dsc), None, P(16), P(16), P(16), P(256), 1 << 20,
+                              None) == mfb.MF_ERR_INVALID_ARG
+    # workspace too small or misaligned
+    need = lib.mf_block_stats_workspace(C.byref(dsc))
+    assert need > 0
+    assert lib.mf_block_stats(C.byref(dsc), P(16), P(16), P(16), P(16), P(256), need - 1,
+                              None) == mfb.MF_ERR_WORKSPACE
+    assert lib.mf_block_stats(C.byref(dsc), P(16), P(16), P(16), P(16), P(257), need,
+                              None) == mfb.MF_ERR_WORKSPACE
+    # select: tau must be positive; cache must match the descriptor
+    cache = mfb.CsrCache(8, 36, 16, 16, 16, 16, 16, 4, 64, mfb.MF_F32, 1, 0x1000)
+    ws = lib.mf_select_extract_workspace(C.byref(dsc))
+    assert lib.mf_select_extract(C.byref(dsc), P(16), P(16), P(16), P(16), 0.0,
+                                 C.byref(cache), P(256), ws, None) == mfb.MF_ERR_INVALID_ARG
+    bad = mfb.CsrCache(8, 36, 16, 16, 16, 16, 16, 5, 64, mfb.MF_F32, 1, 0x1000)
+    assert lib.mf_select_extract(C.byref(dsc), P(16), P(16), P(16), P(16), 0.9,
+                                 C.byref(bad), P(256), ws, None) == mfb.MF_ERR_INVALID_ARG
+    wrong_rows = mfb.CsrCache(9, 36, 16, 16, 16, 16, 16, 4, 64, mfb.MF_F32, 1, 0x1000)
+    assert lib.mf_select_extract(C.byref(dsc), P(16), P(16), P(16), P(16), 0.9,
+                                 C.byref(wrong_rows), P(256), ws, None) == mfb.MF_ERR_INVALID_ARG
+    # mapped AV: Hr must be a multiple of Hkv; page size rule
+    v = mfb.VDesc(16, None, 16, 0, 3, 64)
+    assert lib.mf_mapped_av(C.byref(cache), C.byref(dsc), 4, P(16), C.byref(v), P(16),
+                            None) == mfb.MF_ERR_INVALID_ARG
+    v = mfb.VDesc(16, 16, 8, 64, 2, 64)
+    assert lib.mf_mapped_av(C.byref(cache), C.byref(dsc), 4, P(16), C.byref(v), P(16),
+                            None) == mfb.MF_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------- prefix hashing
+
+def test_prefix_hash_chains_over_the_prefix(lib):
+    rng = np.random.default_rng(2)
+    toks = rng.integers(0, 150000, size=1000).astype(np.int32)
+    h = mfb.prefix_hash(toks, 64)
+    assert h.shape == (16, 2)
+    assert len({tuple(x) for x in h}) == 16
+    np.testing.assert_array_equal(h, mfb.prefix_hash(toks, 64))
+    # a prefix hashes to the same leading blocks
+    np.testing.assert_array_equal(mfb.prefix_hash(toks[:640], 64), h[:10])
+    # changing token 300 changes block 4 and every later block, not earlier ones
+    t2 = toks.copy()
+    t2[300] += 1
+    h2 = mfb.prefix_hash(t2, 64)
+    np.testing.assert_array_equal(h2[:4], h[:4])
+    assert np.all(h2[4:, 0] != h[4:, 0]) and np.all(h2[4:, 1] != h[4:, 1])
+    # the seed changes everything; swapping two tokens in a block changes it
+    assert np.all(mfb.prefix_hash(toks, 64, seed=1) != h)
+    t3 = toks.copy()
+    t3[[5, 6]] = t3[[6, 5]]
+    assert np.all(mfb.prefix_hash(t3, 64)[:, 0] != h[:, 0])
+
+
+def test_index_longest_prefix_and_misses(lib):
+    rng = np.random.default_rng(3)
+    ctx = rng.integers(0, 1000, size=640).astype(np.int32)
+    h = mfb.prefix_hash(ctx, 64)
+    ix = mfb.PrefixIndex()
+    c0 = mfb.CsrCache(10, 55, 0x10, 0x20, 0x30, 0x40, 0x50, 4, 64, mfb.MF_BF16, 1, 0x60)
+    ix.insert(h, sender_layer=3, seq=0, cache_struct=c0)
+    assert len(ix) == 10
+    # a receiver context sharing 6 blocks and then diverging
+    q = np.concatenate([ctx[:400], rng.integers(1000, 2000, size=300).astype(np.int32)])
+    got = ix.lookup(mfb.prefix_hash(q, 64), 3)
+    assert got is not None
+    cache, seq, matched = got
+    assert matched == 6 and seq == 0 and cache.values == 0x50 and cache.row_ptr == 0x10
+    # the full context matches every block; other layer or other text misses
+    assert ix.lookup(h, 3)[2] == 10
+    assert ix.lookup(h, 4) is None
+    assert ix.lookup(mfb.prefix_hash(ctx[::-1].copy(), 64), 3) is None
+    assert ix.lookup(h[:0], 3) is None
+
+
+def test_index_same_key_newest_wins(lib):
+    """Two states under one key (a forced collision): the newer one is kept."""
+    h = mfb.prefix_hash(np.arange(256, dtype=np.int32), 64)
+    ix = mfb.PrefixIndex()
+    a = mfb.CsrCache(4, 10, 1, 2, 3, 4, 5, 4, 64, mfb.MF_BF16, 1, 6)
+    b = mfb.CsrCache(4, 10, 11, 12, 13, 14, 15, 4, 64, mfb.MF_BF16, 2, 16)
+    ix.insert(h, 0, 0, a)
+    ix.insert(h, 0, 1, b)
+    cache, seq, matched = ix.lookup(h, 0)
+    assert (cache.values, seq, matched) == (15, 1, 4)
+    assert len(ix) == 4

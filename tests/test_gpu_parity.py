@@ -1,0 +1,167 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Small cases are compared on every query block (several tiles, ragged tails,
+empty sequences); the full-size workloads are compared on sampled query
+blocks that the oracle computes one by one, in the same launch configuration
+the benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+from cross_model_attention_block_b200 import mapflow as mfb
+from cross_model_attention_block_b200 import synth
+from tests import parity as par
+
+pytestmark = pytest.mark.gpu
+
+
+def _ctx_of(w, dtype=None):
+    dt = dtype or w.torch_dtype
+    return mfb.Context.make(w.lengths, w.Hs, w.d, w.B, w.band_bias, w.band_width, dt)
+
+
+def _small(lengths, Hs, Hr, Hkv, d, B, tau, dtype="bf16", band_bias=2.0, band_width=256,
+           seed=0):
+    w, x = synth.small_case(lengths, Hs, Hr, Hkv, d, B, tau, dtype=dtype, band_bias=band_bias,
+                            band_width=band_width, seed=seed)
+    ctx = _ctx_of(w)
+    gpu = par.run_gpu(ctx, x.Q.cuda(), x.K.cuda(), x.V.cuda(), x.W.cuda(), Hkv, tau)
+    return w, x, ctx, gpu
+
+
+@pytest.mark.parametrize("case", [
+    dict(lengths=[300, 1000, 64, 129, 1], Hs=8, Hr=8, Hkv=2, d=128, B=64, tau=0.9),
+    dict(lengths=[1000, 130], Hs=40, Hr=32, Hkv=8, d=128, B=128, tau=0.95),
+    dict(lengths=[700], Hs=32, Hr=32, Hkv=8, d=128, B=64, tau=0.95),
+    dict(lengths=[333, 65], Hs=4, Hr=4, Hkv=4, d=64, B=64, tau=0.9),
+    dict(lengths=[200, 77], Hs=3, Hr=6, Hkv=3, d=128, B=128, tau=0.9, dtype="f32"),
+    dict(lengths=[100, 0, 70], Hs=5, Hr=4, Hkv=2, d=64, B=64, tau=0.8, dtype="f32"),
+], ids=["bf16_b64_varlen", "bf16_b128_hs40", "bf16_b64_hs32", "bf16_d64",
+        "f32_d128_b128", "f32_empty_seq"])
+def test_small_cases_every_block(case):
+    w, x, ctx, gpu = _small(**case)
+    dt = w.torch_dtype
+    n, ex, worst = par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, gpu,
+                                            par.all_picks(ctx), dt)
+    assert ex <= max(1, n // 50)
+
+
+def test_tiny_f32_workload_every_block():
+    w = synth.workloads()["tiny_f32_n512"]
+    x = synth.single_layer(w)
+    ctx = _ctx_of(w)
+    gpu = par.run_gpu(ctx, x.Q.cuda(), x.K.cuda(), x.V.cuda(), x.W.cuda(), w.Hkv, w.tau)
+    n, ex, worst = par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, gpu,
+                                            par.all_picks(ctx), torch.float32)
+    assert n == 8 and ex == 0 and worst <= 1e-4
+
+
+def test_tau_one_keeps_every_causal_block():
+    w, x, ctx, gpu = _small([260, 64], 4, 4, 2, 128, 64, 1.0)
+    cache = gpu[2]
+    nqb, nblocks = ctx.layout_sizes()
+    assert cache.nnz == nblocks
+    rp, ci = par.kept_sets(cache)
+    g = 0
+    for L in (260, 64):
+        for qb in range((L + 63) // 64):
+            assert list(ci[rp[g]:rp[g + 1]]) == list(range(qb + 1))
+            g += 1
+
+
+def test_capacity_overflow_is_reported():
+    w, x = synth.small_case([400], 4, 4, 2, 128, 64, 0.99)
+    ctx = _ctx_of(w)
+    Q, K = x.Q.cuda(), x.K.cuda()
+    lse, mass = mfb.block_stats(ctx, Q, K)
+    cache = mfb.Cache(ctx, capacity=5)
+    mfb.select_extract(ctx, Q, K, lse, mass, 0.99, cache=cache)
+    mfb.mapped_av(cache, 4, x.W.cuda(), x.V.cuda(), 2)
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.sync_status()
+    assert e.value.status == mfb.MF_ERR_CAPACITY
+    mfb.sync_status()  # the status word was cleared by the read
+
+
+def test_mid_workload_every_block():
+    w = synth.workloads()["mid_bf16_n8192"]
+    x = synth.single_layer(w)
+    ctx = _ctx_of(w)
+    gpu = par.run_gpu(ctx, x.Q.cuda(), x.K.cuda(), x.V.cuda(), x.W.cuda(), w.Hkv, w.tau)
+    picks = par.all_picks(ctx)
+    n, ex, worst = par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, gpu,
+                                            picks, torch.bfloat16, check_values=False)
+    assert n == 128 and ex <= 2
+    # extracted values on a subset
+    par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, gpu,
+                             [(0, 0), (0, 1), (0, 63), (0, 127)], torch.bfloat16)
+
+
+def test_large_workload_sampled():
+    w = synth.workloads()["large_bf16_n32768"]
+    x = synth.single_layer(w)
+    ctx = _ctx_of(w)
+    gpu = par.run_gpu(ctx, x.Q.cuda(), x.K.cuda(), x.V.cuda(), x.W.cuda(), w.Hkv, w.tau)
+    picks = [(0, 0), (0, 1), (0, 2), (0, 77), (0, 128), (0, 254), (0, 255)]
+    n, ex, worst = par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, gpu,
+                                            picks, torch.bfloat16)
+    assert ex <= 1
+    # properties that hold at any size: every row keeps its diagonal block, the
+    # row pointers are consistent, every output is finite
+    cache, O = gpu[2], gpu[3]
+    rp, ci = par.kept_sets(cache)
+    nqb = 256
+    assert rp[0] == 0 and np.all(np.diff(rp) >= 1) and rp[-1] == cache.nnz
+    for g in range(nqb):
+        row = ci[rp[g]:rp[g + 1]]
+        assert row[-1] == g and np.all(np.diff(row) > 0)
+    assert torch.isfinite(O.float()).all()
+
+
+def test_multi_receiver_share_one_sender_cache():
+    """One compressed sender layer feeds receiver layers of two receivers."""
+    w = synth.workloads()["multi_receiver_n16384"]
+    ctx = _ctx_of(w)
+    caches = {}
+    sender = {}
+    for sl in (0, 2):
+        Q, K = synth.sender_layer(w, sl)
+        sender[sl] = (Q, K)
+        Qd, Kd = Q.cuda(), K.cuda()
+        lse, mass = mfb.block_stats(ctx, Qd, Kd)
+        caches[sl] = (mfb.select_extract(ctx, Qd, Kd, lse, mass, w.tau), lse, mass)
+    for rec, (name, nl, table) in enumerate(w.receivers):
+        for layer in range(nl):
+            sl = table[layer]
+            if sl not in caches:
+                continue
+            V, W = synth.receiver_layer(w, rec, layer)
+            cache, lse, mass = caches[sl]
+            O = mfb.mapped_av(cache, w.Hr, W.cuda(), V.cuda(), w.Hkv)
+            mfb.sync_status()
+            Q, K = sender[sl]
+            gpu = (lse, mass, cache, O)
+            par.compare_query_blocks(ctx, Q, K, V, W, w.Hkv, w.tau, gpu,
+                                     [(0, 0), (0, 100), (0, 255)], torch.bfloat16,
+                                     check_values=False)
+
+
+def test_varlen_paged_workload_sampled():
+    w = synth.workloads()["varlen_paged_64seq"]
+    x = synth.single_layer(w)
+    pool, table = synth.paged_v(x.V, w.lengths, synth.page_rng(w))
+    ctx = _ctx_of(w)
+    Q, K = x.Q.cuda(), x.K.cuda()
+    gpu = par.run_gpu(ctx, Q, K, None, x.W.cuda(), w.Hkv, w.tau, page_table=table.cuda(),
+                      Vpool=pool.cuda())
+    lens = np.array(w.lengths)
+    longest, shortest = int(np.argmax(lens)), int(np.argmin(lens))
+    picks = [(0, 0), (shortest, (lens[shortest] - 1) // 64), (longest, (lens[longest] - 1) // 64),
+             (longest, 100), (17, 5), (63, (lens[63] - 1) // 64)]
+    par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, gpu, picks,
+                             torch.bfloat16)
+    # paged V gives exactly the contiguous result
+    O_c = mfb.mapped_av(gpu[2], w.Hr, x.W.cuda(), x.V.cuda(), w.Hkv)
+    mfb.sync_status()
+    assert torch.equal(O_c, gpu[3])

@@ -79,14 +79,19 @@ static mf_status check_desc(const mf_attn_desc* d, Sizes* sz) {
   return MF_OK;
 }
 
-static size_t meta_bytes(Carve& c, int nseq, Meta* m) {
+static size_t meta_bytes(Carve& c, int nseq, int64_t ntiles, Meta* m) {
   Meta mm;
   mm.cu_qb = c.take<int32_t>(nseq + 1);
   mm.cu_blk = c.take<int64_t>(nseq + 1);
   mm.cu_tile = c.take<int32_t>(nseq + 1);
+  mm.tiles = c.take<int32_t>(2 * size_t(ntiles) + 2);
   if (m) *m = mm;
   return c.used;
 }
+
+// bf16 with d = 128 runs on the tcgen05 kernels; float32 (1e-4 relative
+// accuracy) and d = 64 run on the scalar kernels.
+static bool use_tc(const mf_attn_desc& d) { return d.dt == MF_BF16 && d.d == 128; }
 
 static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
 
@@ -95,7 +100,7 @@ static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) &
 static size_t stats_ws(const mf_attn_desc& d, const Sizes& sz, void* base, Meta* m,
                        float** part) {
   Carve c(base);
-  meta_bytes(c, d.nseq, m);
+  meta_bytes(c, d.nseq, sz.ntiles, m);
   float* p = c.take<float>(size_t(d.Hs) * size_t(sz.nblocks));
   if (part) *part = p;
   return c.used + 256;
@@ -104,7 +109,7 @@ static size_t stats_ws(const mf_attn_desc& d, const Sizes& sz, void* base, Meta*
 static size_t select_ws(const mf_attn_desc& d, const Sizes& sz, void* base, Meta* m,
                         int32_t** counts, uint8_t** keep, int32_t** slot) {
   Carve c(base);
-  meta_bytes(c, d.nseq, m);
+  meta_bytes(c, d.nseq, sz.ntiles, m);
   int32_t* a = c.take<int32_t>(size_t(sz.nqb) + 1);
   uint8_t* b = c.take<uint8_t>(size_t(sz.nblocks) + 1);
   int32_t* s = c.take<int32_t>(size_t(sz.nblocks) + 1);
@@ -157,7 +162,8 @@ mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
   cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, m, s);
   if (e != cudaSuccess) return cuda_fail(e, "meta");
   if (sz.nqb == 0) return MF_OK;
-  e = launch_stats_simt(d, sz, m, Q, K, lse, part, s);
+  e = use_tc(d) ? launch_stats_tc(d, sz, m, Q, K, lse, part, s)
+                : launch_stats_simt(d, sz, m, Q, K, lse, part, s);
   if (e != cudaSuccess) return cuda_fail(e, "block stats");
   e = launch_mass_reduce(part, d.Hs, sz.nblocks, mass, s);
   if (e != cudaSuccess) return cuda_fail(e, "mass reduce");
@@ -211,7 +217,8 @@ mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void*
   }
   e = launch_select(d, sz, m, mass, tau, *out, counts, keep, slot, s);
   if (e != cudaSuccess) return cuda_fail(e, "select");
-  e = launch_extract_simt(d, sz, Q, K, lse, *out, s);
+  e = use_tc(d) ? launch_extract_tc(d, sz, m, Q, K, lse, slot, out->values, s)
+                : launch_extract_simt(d, sz, Q, K, lse, *out, s);
   if (e != cudaSuccess) return cuda_fail(e, "extract");
   return MF_OK;
 }

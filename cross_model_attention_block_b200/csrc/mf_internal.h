@@ -20,6 +20,7 @@ struct Meta {
   int32_t* cu_qb;    // [nseq+1] prefix of ceil(L_s/B)
   int64_t* cu_blk;   // [nseq+1] prefix of C_s
   int32_t* cu_tile;  // [nseq+1] prefix of ceil(L_s/128)
+  int32_t* tiles;    // [ntiles][2] (sequence, 128-row tile), longest causal rows first
 };
 
 // Host-side sizes of a context.
@@ -48,6 +49,14 @@ struct Carve {
 // ---- launchers (return cudaGetLastError of the launch) ----
 cudaError_t launch_meta(int nseq, const int32_t* cu_seqlens, int B, const Meta& m,
                         cudaStream_t st);
+
+// Tensor-core kernels (bf16, d = 128).
+cudaError_t launch_stats_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
+                            const void* Q, const void* K, float* lse, float* part,
+                            cudaStream_t st);
+cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
+                              const void* Q, const void* K, const float* lse,
+                              const int32_t* slot, void* values, cudaStream_t st);
 
 cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                               const void* Q, const void* K, float* lse, float* part,

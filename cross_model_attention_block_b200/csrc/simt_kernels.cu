@@ -21,9 +21,9 @@ namespace mf {
 // ---------------------------------------------------------------- metadata
 
 __global__ void k_meta(int nseq, const int32_t* __restrict__ cu_seqlens, int B, int32_t* cu_qb,
-                       int64_t* cu_blk, int32_t* cu_tile) {
+                       int64_t* cu_blk, int32_t* cu_tile, int32_t* tiles) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int32_t q = 0, t = 0;
+  int32_t q = 0, t = 0, tmax = 0;
   int64_t b = 0;
   cu_qb[0] = 0;
   cu_blk[0] = 0;
@@ -31,18 +31,29 @@ __global__ void k_meta(int nseq, const int32_t* __restrict__ cu_seqlens, int B, 
   for (int s = 0; s < nseq; ++s) {
     int L = cu_seqlens[s + 1] - cu_seqlens[s];
     int n = (L + B - 1) / B;
+    int nt = (L + 127) / 128;
     q += n;
     b += int64_t(n) * (n + 1) / 2;
-    t += (L + 127) / 128;
+    t += nt;
+    tmax = max(tmax, nt);
     cu_qb[s + 1] = q;
     cu_blk[s + 1] = b;
     cu_tile[s + 1] = t;
   }
+  // 128-row tiles ordered by tile index descending (longest causal rows first)
+  int w = 0;
+  for (int tt = tmax - 1; tt >= 0; --tt)
+    for (int s = 0; s < nseq; ++s)
+      if (tt < cu_tile[s + 1] - cu_tile[s]) {
+        tiles[2 * w] = s;
+        tiles[2 * w + 1] = tt;
+        ++w;
+      }
 }
 
 cudaError_t launch_meta(int nseq, const int32_t* cu_seqlens, int B, const Meta& m,
                         cudaStream_t st) {
-  k_meta<<<1, 32, 0, st>>>(nseq, cu_seqlens, B, m.cu_qb, m.cu_blk, m.cu_tile);
+  k_meta<<<1, 32, 0, st>>>(nseq, cu_seqlens, B, m.cu_qb, m.cu_blk, m.cu_tile, m.tiles);
   return cudaGetLastError();
 }
 

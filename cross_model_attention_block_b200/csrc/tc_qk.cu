@@ -1,0 +1,459 @@
+// Tensor-core (tcgen05 + TMA) kernels over the causal sender logits, bf16, d = 128.
+//
+// MapFlow article (163.com, section on the three system components): the
+// sender's attention map is compressed in stages -- block-level statistics
+// first, then extraction of the kept blocks -- never forming the dense N x N
+// matrix.  Both stages walk the causal QK^T of one (head, 128-row query tile)
+// pair tile by tile; they differ only in what the epilogue does with a tile.
+//
+//  * Block statistics (one pass): online row max and sum give the row
+//    log-sum-exp; each key block's partial sum is kept as a log value
+//    a = m + log2(sum_j 2^(x_j - m)) in TMEM columns 256.., so that after the
+//    last tile mass contribution = 2^(a - lse2) needs no second QK^T pass.
+//  * Extraction: for every kept block of the tile, P = 2^(x - lse2) rounded to
+//    bf16 and written in the cache layout.
+//
+// Roles (256 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// tcgen05.mma from one thread, warps 4..7 (one per TMEM lane quarter, one
+// query row per thread) run the epilogue.  S = Q K^T for a 128 x 128 tile
+// lands in one of two TMEM buffers (columns 0..255) so the next tile's MMA
+// overlaps this tile's epilogue; K tiles stream through a 4-stage ring.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "mf_sm100.cuh"
+
+namespace mf {
+using namespace sm100;
+
+namespace qk {
+
+constexpr int kTile = 128;
+constexpr int kD = 128;
+constexpr int kStages = 4;
+constexpr int kThreads = 256;
+constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB: two [128][64] swizzled halves
+constexpr uint32_t kHalfBytes = kTileBytes / 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAcol = 256;  // first TMEM column of the per-key-block log partials
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+enum Mode { kStats = 0, kExtract = 1 };
+
+struct Smem {
+  uint8_t q[kTileBytes];
+  uint8_t k[kStages][kTileBytes];
+  float red[4][32];
+  uint64_t q_full;
+  uint64_t k_full[kStages];
+  uint64_t k_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t s_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+};
+
+struct Params {
+  const int32_t* cu_seqlens;
+  const int32_t* tiles;    // [ntiles][2] = (sequence, 128-row tile), heaviest first
+  const int64_t* cu_blk;   // [nseq+1]
+  const int32_t* cu_qb;    // [nseq+1]
+  int ntiles;
+  int Hs;
+  int B;
+  int band_width;
+  float scale2;            // log2(e) / sqrt(d)
+  float bias2;             // band_bias * log2(e)
+  int64_t ntok;
+  int64_t nblocks;
+  float* lse;              // stats: out [Hs][ntok] (natural log); extract: in
+  float* part;             // stats: out [Hs][nblocks]
+  const int32_t* slot;     // extract: block -> cache entry or -1
+  __nv_bfloat16* values;   // extract: out
+  unsigned* status;
+};
+
+// Does key tile kt of query tile t hold a kept block (extract) -- every
+// causal key tile counts for the statistics.
+template <int MODE, int BB>
+__device__ __forceinline__ bool tile_needed(const Params& p, int s, int t, int kt, int nqb_s) {
+  if (MODE == kStats) return true;
+  const int64_t cb = p.cu_blk[s];
+  if (BB == 128) {
+    return p.slot[cb + int64_t(t) * (t + 1) / 2 + kt] >= 0;
+  }
+  for (int a = 0; a < 2; ++a) {
+    int qb = 2 * t + a;
+    if (qb >= nqb_s) break;
+    for (int b = 0; b < 2; ++b) {
+      int kb = 2 * kt + b;
+      if (kb <= qb && p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kb] >= 0) return true;
+    }
+  }
+  return false;
+}
+
+// Lane l ends up holding sum over the warp of v[l] (v has 32 entries).
+__device__ __forceinline__ float transpose_reduce32(float* v, int lane) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int k = 0; k < s; ++k) {
+      float send = upper ? v[k] : v[k + s];
+      float keep = upper ? v[k + s] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ void named_sync_epilogue() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// AND of a predicate over the 128 epilogue threads (named barrier 1).
+__device__ __forceinline__ bool epilogue_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v))
+      : "memory");
+  return r != 0;
+}
+
+template <int MODE, int BB>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_qk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+         const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                      ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x / p.ntiles;
+  const int w = blockIdx.x % p.ntiles;
+  const int s = p.tiles[2 * w], t = p.tiles[2 * w + 1];
+  const int seq0 = p.cu_seqlens[s];
+  const int L = p.cu_seqlens[s + 1] - seq0;
+  const int nqb_s = p.cu_qb[s + 1] - p.cu_qb[s];
+  const int row0 = t * kTile;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm.k_full[i], 1);
+      mbar_init(&sm.k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_empty[i], 128);
+    }
+    mbar_init(&sm.drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      mbar_expect_tx(&sm.q_full, kTileBytes);
+      tma_load_2d(sm.q, &tmQ, &sm.q_full, h * kD, seq0 + row0);
+      tma_load_2d(sm.q + kHalfBytes, &tmQ, &sm.q_full, h * kD + 64, seq0 + row0);
+      int n = 0;
+      for (int kt = 0; kt <= t; ++kt) {
+        if (!tile_needed<MODE, BB>(p, s, t, kt, nqb_s)) continue;
+        const int st = n % kStages;
+        if (!mbar_wait(&sm.k_empty[st], ((n / kStages) & 1) ^ 1, p.status)) break;
+        mbar_expect_tx(&sm.k_full[st], kTileBytes);
+        tma_load_2d(sm.k[st], &tmK, &sm.k_full[st], h * kD, seq0 + kt * kTile);
+        tma_load_2d(sm.k[st] + kHalfBytes, &tmK, &sm.k_full[st], h * kD + 64,
+                    seq0 + kt * kTile);
+        ++n;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 0);
+      const uint32_t q_addr = smem_u32(sm.q);
+      bool ok = mbar_wait(&sm.q_full, 0, p.status);
+      int n = 0;
+      for (int kt = 0; ok && kt <= t; ++kt) {
+        if (!tile_needed<MODE, BB>(p, s, t, kt, nqb_s)) continue;
+        const int st = n % kStages, sb = n & 1;
+        if (!mbar_wait(&sm.k_full[st], (n / kStages) & 1, p.status)) break;
+        if (!mbar_wait(&sm.s_empty[sb], ((n >> 1) & 1) ^ 1, p.status)) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sm.k[st]);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          mma_bf16_ss(tmem + sb * 128, smem_desc(q_addr + off, 16, 1024, kSwizzle128),
+                      smem_desc(k_addr + off, 16, 1024, kSwizzle128), idesc, kk > 0);
+        }
+        mma_commit(&sm.k_empty[st]);
+        mma_commit(&sm.s_full[sb]);
+        ++n;
+      }
+      // every MMA issued above has completed once this arrives
+      mma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, p.status);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // tile row
+    const int ri = row0 + r;            // row within the sequence
+    const bool valid = ri < L;
+    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
+    const int W = p.band_width;
+    float m_run = -CUDART_INF_F, l_run = 0.f;
+    float lse2 = 0.f;
+    if (MODE == kExtract) lse2 = valid ? p.lse[int64_t(h) * p.ntok + seq0 + ri] * kLog2e : 0.f;
+    const int qb_r = (BB == 128) ? t : 2 * t + (r >> 6);
+    const int64_t cb = p.cu_blk[s];
+    int n = 0;
+    bool ok = true;
+    for (int kt = 0; kt <= t; ++kt) {
+      if (!tile_needed<MODE, BB>(p, s, t, kt, nqb_s)) continue;
+      const int sb = n & 1;
+      if (!mbar_wait(&sm.s_full[sb], (n >> 1) & 1, p.status)) { ok = false; break; }
+      tc_fence_after();
+      float v[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + sb * 128 + c * 32, v + c * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&sm.s_empty[sb]);
+
+      // logits in log2 units with band bias and causal mask
+      const int kbase = kt * kTile;
+      const bool band_tile = (row0 + kTile - 1) - kbase >= 0 && row0 - (kbase + kTile - 1) < W;
+      const bool diag = kt == t;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const int j = kbase + c;
+        float x = v[c] * p.scale2;
+        if (band_tile && ri - j < W) x += p.bias2;
+        if (diag && j > ri) x = -CUDART_INF_F;
+        v[c] = x;
+      }
+      if (MODE == kStats) {
+        float mt = -CUDART_INF_F;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mt = fmaxf(mt, v[c]);
+        const float m_new = valid ? fmaxf(m_run, mt) : 0.f;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s0 += ex2(v[c] - m_new);
+#pragma unroll
+        for (int c = 64; c < 128; ++c) s1 += ex2(v[c] - m_new);
+        l_run = l_run * ex2(m_run - m_new) + s0 + s1;
+        m_run = m_new;
+        if (BB == 128) {
+          float a = valid ? m_new + lg2(s0 + s1) : -CUDART_INF_F;
+          tmem_st1(lane_addr + kAcol + kt, a);
+        } else {
+          float a0 = valid ? m_new + lg2(s0) : -CUDART_INF_F;
+          float a1 = valid ? m_new + lg2(s1) : -CUDART_INF_F;
+          tmem_st2(lane_addr + kAcol + 2 * kt, a0, a1);
+        }
+      } else {
+        // extraction of the kept blocks of this tile that contain row ri
+        constexpr int nkb_tile = kTile / BB;
+#pragma unroll
+        for (int b = 0; b < nkb_tile; ++b) {
+          const int kb = kt * nkb_tile + b;
+          if (kb > qb_r) continue;
+          const int64_t e = p.slot[cb + int64_t(qb_r) * (qb_r + 1) / 2 + kb];
+          if (e < 0) continue;
+          const int il = ri - qb_r * BB;
+          const int swap = ((h >> 2) & 1) ? 8 : 0;
+#pragma unroll
+          for (int g = 0; g < BB / 16; ++g) {
+            __align__(16) __nv_bfloat16 o[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              float x = v[b * BB + g * 16 + k];
+              o[k ^ swap] = __float2bfloat16_rn(valid ? ex2(x - lse2) : 0.f);
+            }
+            __nv_bfloat16* dst =
+                p.values + ((((e * (BB >> 4) + g) * BB + il) * p.Hs + h) << 4);
+            reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(o)[0];
+            reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(o)[1];
+          }
+        }
+      }
+      ++n;
+    }
+    ok = epilogue_all(ok);  // uniform, so every thread takes the named barriers below
+    if (MODE == kStats && ok) {
+      lse2 = valid ? m_run + lg2(l_run) : 0.f;
+      if (valid) p.lse[int64_t(h) * p.ntok + seq0 + ri] = lse2 * kLn2;
+      tmem_wait_st();
+      const int nkb = (t + 1) * (kTile / BB);
+      for (int c0 = 0; c0 < nkb; c0 += 32) {
+        float a[32];
+        tmem_ld32(lane_addr + kAcol + c0, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          a[k] = (valid && c0 + k < nkb) ? ex2(a[k] - lse2) : 0.f;
+        const float tot = transpose_reduce32(a, lane);
+        named_sync_epilogue();
+        sm.red[quarter][lane] = tot;
+        named_sync_epilogue();
+        if (quarter == 0) {
+          const int kb = c0 + lane;
+          if (BB == 128) {
+            float m = (sm.red[0][lane] + sm.red[1][lane]) + (sm.red[2][lane] + sm.red[3][lane]);
+            if (kb <= t) p.part[int64_t(h) * p.nblocks + cb + int64_t(t) * (t + 1) / 2 + kb] = m;
+          } else {
+            const int qa = 2 * t, qbb = 2 * t + 1;
+            float m0 = sm.red[0][lane] + sm.red[1][lane];
+            float m1 = sm.red[2][lane] + sm.red[3][lane];
+            if (kb <= qa) p.part[int64_t(h) * p.nblocks + cb + int64_t(qa) * (qa + 1) / 2 + kb] = m0;
+            if (qbb < nqb_s && kb <= qbb)
+              p.part[int64_t(h) * p.nblocks + cb + int64_t(qbb) * (qbb + 1) / 2 + kb] = m1;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------- host side
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+}  // namespace qk
+
+static qk::EncodeTiled encode_fn() {
+  static qk::EncodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<qk::EncodeTiled>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over rows x cols (cols contiguous), box {64, box_rows},
+// 128-byte swizzle.
+cudaError_t make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                              uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+  qk::EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_3d_bf16(CUtensorMap* m, const void* base, const uint64_t dims[3],
+                              const uint64_t strides_bytes[2], const uint32_t box[3],
+                              bool swizzle128) {
+  qk::EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides_bytes[0], strides_bytes[1]};
+  cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), d, st, bx,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, const Meta& m,
+                             const void* Q, const void* K, float* lse, float* part,
+                             const int32_t* slot, void* values, cudaStream_t st) {
+  if (sz.ntiles == 0) return cudaSuccess;
+  CUtensorMap tq, tk;
+  const uint64_t cols = uint64_t(d.Hs) * d.d;
+  cudaError_t e = make_tmap_2d_bf16(&tq, Q, uint64_t(sz.ntok), cols, 64, qk::kTile, true);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_2d_bf16(&tk, K, uint64_t(sz.ntok), cols, 64, qk::kTile, true);
+  if (e != cudaSuccess) return e;
+  qk::Params p{};
+  p.cu_seqlens = d.cu_seqlens;
+  p.tiles = m.tiles;
+  p.cu_blk = m.cu_blk;
+  p.cu_qb = m.cu_qb;
+  p.ntiles = int(sz.ntiles);
+  p.Hs = d.Hs;
+  p.B = d.B;
+  p.band_width = d.band_width;
+  p.scale2 = qk::kLog2e / sqrtf(float(d.d));
+  p.bias2 = d.band_bias * qk::kLog2e;
+  p.ntok = sz.ntok;
+  p.nblocks = sz.nblocks;
+  p.lse = lse;
+  p.part = part;
+  p.slot = slot;
+  p.values = static_cast<__nv_bfloat16*>(values);
+  p.status = status_word();
+  const size_t smem = sizeof(qk::Smem) + 1024;
+  const unsigned grid = unsigned(sz.ntiles) * unsigned(d.Hs);
+#define MF_QK(MODE, BB)                                                                       \
+  do {                                                                                        \
+    e = cudaFuncSetAttribute(qk::k_qk<MODE, BB>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             int(smem));                                                      \
+    if (e != cudaSuccess) return e;                                                           \
+    qk::k_qk<MODE, BB><<<grid, qk::kThreads, smem, st>>>(tq, tk, p);                          \
+  } while (0)
+  if (mode == qk::kStats) {
+    if (d.B == 128) MF_QK(qk::kStats, 128); else MF_QK(qk::kStats, 64);
+  } else {
+    if (d.B == 128) MF_QK(qk::kExtract, 128); else MF_QK(qk::kExtract, 64);
+  }
+#undef MF_QK
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
+                            const void* Q, const void* K, float* lse, float* part,
+                            cudaStream_t st) {
+  return launch_qk(qk::kStats, d, sz, m, Q, K, lse, part, nullptr, nullptr, st);
+}
+
+cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
+                              const void* Q, const void* K, const float* lse,
+                              const int32_t* slot, void* values, cudaStream_t st) {
+  return launch_qk(qk::kExtract, d, sz, m, Q, K, const_cast<float*>(lse), nullptr, slot,
+                   values, st);
+}
+
+}  // namespace mf

@@ -162,7 +162,9 @@ mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
   cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, m, s);
   if (e != cudaSuccess) return cuda_fail(e, "meta");
   if (sz.nqb == 0) return MF_OK;
-  e = use_tc(d) ? launch_stats_tc(d, sz, m, Q, K, lse, part, s)
+  // the one-pass statistics keep one TMEM column per key block: 256 at most
+  const bool tc_stats = use_tc(d) && (sz.max_len + d.B - 1) / d.B <= 256;
+  e = tc_stats ? launch_stats_tc(d, sz, m, Q, K, lse, part, s)
                 : launch_stats_simt(d, sz, m, Q, K, lse, part, s);
   if (e != cudaSuccess) return cuda_fail(e, "block stats");
   e = launch_mass_reduce(part, d.Hs, sz.nblocks, mass, s);
@@ -217,7 +219,8 @@ mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void*
   }
   e = launch_select(d, sz, m, mass, tau, *out, counts, keep, slot, s);
   if (e != cudaSuccess) return cuda_fail(e, "select");
-  e = use_tc(d) ? launch_extract_tc(d, sz, m, Q, K, lse, slot, out->values, s)
+  e = use_tc(d) ? launch_extract_tc(d, sz, m, Q, K, lse, slot, out->values,
+                                    out->nnz_capacity, s)
                 : launch_extract_simt(d, sz, Q, K, lse, *out, s);
   if (e != cudaSuccess) return cuda_fail(e, "extract");
   return MF_OK;

@@ -29,15 +29,10 @@ __device__ __forceinline__ int upper_index(const I* a, int n, int64_t v) {
   return lo;
 }
 
-// Position of key (j % 16) inside its stored 16-key group for head h: the two
-// 8-key halves are swapped when bit 2 of h is set.  Spreads the eight heads
-// read together by a transposing shared-memory load over all banks.
-__device__ __forceinline__ int key_slot(int j16, int h) { return j16 ^ (((h >> 2) & 1) << 3); }
-
-// Element offset of (entry e, row i, head h, key j) in the CSR value array
-// [nnz][B/16][B][Hs][16].
+// Element offset of (entry e, head h, row i, key j) in the CSR value array
+// [nnz][Hs][B][B].
 __device__ __forceinline__ int64_t value_offset(int64_t e, int i, int h, int j, int B, int Hs) {
-  return (((e * (B >> 4) + (j >> 4)) * B + i) * Hs + h) * 16 + key_slot(j & 15, h);
+  return ((e * Hs + h) * B + i) * int64_t(B) + j;
 }
 
 __device__ __forceinline__ uint64_t global_ns() {

@@ -56,7 +56,8 @@ cudaError_t launch_stats_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& 
                             cudaStream_t st);
 cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                               const void* Q, const void* K, const float* lse,
-                              const int32_t* slot, void* values, cudaStream_t st);
+                              const int32_t* slot, void* values, int64_t capacity,
+                              cudaStream_t st);
 
 cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                               const void* Q, const void* K, float* lse, float* part,

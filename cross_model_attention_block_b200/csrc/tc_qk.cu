@@ -17,12 +17,13 @@
 // tcgen05.mma from one thread, warps 4..7 (one per TMEM lane quarter, one
 // query row per thread) run the epilogue.  S = Q K^T for a 128 x 128 tile
 // lands in one of two TMEM buffers (columns 0..255) so the next tile's MMA
-// overlaps this tile's epilogue; K tiles stream through a 4-stage ring.
+// overlaps this tile's epilogue; K tiles stream through a 3-stage ring.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "mf_sm100.cuh"
@@ -34,7 +35,7 @@ namespace qk {
 
 constexpr int kTile = 128;
 constexpr int kD = 128;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kThreads = 256;
 constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB: two [128][64] swizzled halves
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
@@ -48,6 +49,9 @@ enum Mode { kStats = 0, kExtract = 1 };
 struct Smem {
   uint8_t q[kTileBytes];
   uint8_t k[kStages][kTileBytes];
+  // extraction: two staging tiles for TMA stores, each either two [128][64]
+  // (B = 128) or four [64][64] (B = 64) bf16 sub-tiles, 128-byte swizzled
+  uint8_t out[2][kTileBytes];
   float red[4][32];
   uint64_t q_full;
   uint64_t k_full[kStages];
@@ -134,7 +138,7 @@ __device__ __forceinline__ bool epilogue_all(bool v) {
 template <int MODE, int BB>
 __global__ void __launch_bounds__(kThreads, 1)
     k_qk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-         const Params p) {
+         const __grid_constant__ CUtensorMap tmV, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
@@ -232,7 +236,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int kt = 0; kt <= t; ++kt) {
       if (!tile_needed<MODE, BB>(p, s, t, kt, nqb_s)) continue;
       const int sb = n & 1;
-      if (!mbar_wait(&sm.s_full[sb], (n >> 1) & 1, p.status)) { ok = false; break; }
+      bool got = mbar_wait(&sm.s_full[sb], (n >> 1) & 1, p.status);
+      // extraction takes named barriers inside the loop: leave it together
+      if (MODE == kExtract) got = epilogue_all(got);
+      if (!got) { ok = false; break; }
       tc_fence_after();
       float v[128];
 #pragma unroll
@@ -274,33 +281,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st2(lane_addr + kAcol + 2 * kt, a0, a1);
         }
       } else {
-        // extraction of the kept blocks of this tile that contain row ri
-        constexpr int nkb_tile = kTile / BB;
+        // Extraction.  The tile's kept blocks are staged in out[n & 1] as
+        // 128-byte-swizzled [rows][64 keys] sub-tiles and written by TMA
+        // stores: sub-tile b (keys 64b..) for B = 128, (row half a, key half
+        // b) for B = 64.  A row writes only into blocks of its own query
+        // block (which must exist) that are kept.
+        uint8_t* obuf = sm.out[n & 1];
+        if (threadIdx.x == 128) bulk_wait_read<1>();  // stores of tile n-2 done reading
+        named_sync_epilogue();
+        const int rr = (BB == 128) ? r : (r & 63);
+        const bool row_ok = qb_r < nqb_s;
 #pragma unroll
-        for (int b = 0; b < nkb_tile; ++b) {
-          const int kb = kt * nkb_tile + b;
-          if (kb > qb_r) continue;
-          const int64_t e = p.slot[cb + int64_t(qb_r) * (qb_r + 1) / 2 + kb];
-          if (e < 0) continue;
-          const int il = ri - qb_r * BB;
-          const int swap = ((h >> 2) & 1) ? 8 : 0;
+        for (int b = 0; b < 2; ++b) {
+          const int kb = (BB == 128) ? kt : 2 * kt + b;
+          if (!row_ok || kb > qb_r || p.slot[cb + int64_t(qb_r) * (qb_r + 1) / 2 + kb] < 0)
+            continue;
+          uint8_t* sub = obuf + ((BB == 128) ? b * kHalfBytes : ((r >> 6) * 2 + b) * 8192);
 #pragma unroll
-          for (int g = 0; g < BB / 16; ++g) {
-            __align__(16) __nv_bfloat16 o[16];
+          for (int c = 0; c < 8; ++c) {
+            uint32_t w4[4];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              float x = v[b * BB + g * 16 + k];
-              o[k ^ swap] = __float2bfloat16_rn(valid ? ex2(x - lse2) : 0.f);
+            for (int k = 0; k < 4; ++k) {
+              const float x0 = v[b * 64 + c * 8 + 2 * k], x1 = v[b * 64 + c * 8 + 2 * k + 1];
+              __nv_bfloat162 pr = __floats2bfloat162_rn(valid ? ex2(x0 - lse2) : 0.f,
+                                                        valid ? ex2(x1 - lse2) : 0.f);
+              w4[k] = *reinterpret_cast<uint32_t*>(&pr);
             }
-            __nv_bfloat16* dst =
-                p.values + ((((e * (BB >> 4) + g) * BB + il) * p.Hs + h) << 4);
-            reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(o)[0];
-            reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(o)[1];
+            *reinterpret_cast<uint4*>(sub + rr * 128 + ((c ^ (rr & 7)) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
+        }
+        fence_proxy_async_smem();
+        named_sync_epilogue();
+        if (threadIdx.x == 128) {
+#pragma unroll
+          for (int a = 0; a < kTile / BB; ++a) {
+            const int qb = (BB == 128) ? t : 2 * t + a;
+            if (qb >= nqb_s) continue;
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              const int kb = (BB == 128) ? kt : 2 * kt + b;
+              if (kb > qb) continue;
+              const int64_t e = p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kb];
+              if (e < 0) continue;
+              const uint8_t* sub = obuf + ((BB == 128) ? b * kHalfBytes : (a * 2 + b) * 8192);
+              tma_store_2d(&tmV, sub, (BB == 128) ? b * 64 : 0,
+                           int32_t((e * p.Hs + h) * BB));
+            }
+          }
+          bulk_commit();
         }
       }
       ++n;
     }
+    if (MODE == kExtract && threadIdx.x == 128) bulk_wait_all<0>();
     ok = epilogue_all(ok);  // uniform, so every thread takes the named barriers below
     if (MODE == kStats && ok) {
       lse2 = valid ? m_run + lg2(l_run) : 0.f;
@@ -399,7 +433,8 @@ cudaError_t make_tmap_3d_bf16(CUtensorMap* m, const void* base, const uint64_t d
 
 static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                              const void* Q, const void* K, float* lse, float* part,
-                             const int32_t* slot, void* values, cudaStream_t st) {
+                             const int32_t* slot, void* values, int64_t capacity,
+                             cudaStream_t st) {
   if (sz.ntiles == 0) return cudaSuccess;
   CUtensorMap tq, tk;
   const uint64_t cols = uint64_t(d.Hs) * d.d;
@@ -407,6 +442,14 @@ static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, c
   if (e != cudaSuccess) return e;
   e = make_tmap_2d_bf16(&tk, K, uint64_t(sz.ntok), cols, 64, qk::kTile, true);
   if (e != cudaSuccess) return e;
+  CUtensorMap tv;  // the cache values as [capacity * Hs * B rows][B keys] (extraction only)
+  memset(&tv, 0, sizeof(tv));
+  if (mode == qk::kExtract) {
+    if (capacity < 1) return cudaSuccess;
+    e = make_tmap_2d_bf16(&tv, values, uint64_t(capacity) * d.Hs * d.B, uint64_t(d.B), 64,
+                          uint32_t(d.B), true);
+    if (e != cudaSuccess) return e;
+  }
   qk::Params p{};
   p.cu_seqlens = d.cu_seqlens;
   p.tiles = m.tiles;
@@ -432,7 +475,7 @@ static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, c
     e = cudaFuncSetAttribute(qk::k_qk<MODE, BB>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              int(smem));                                                      \
     if (e != cudaSuccess) return e;                                                           \
-    qk::k_qk<MODE, BB><<<grid, qk::kThreads, smem, st>>>(tq, tk, p);                          \
+    qk::k_qk<MODE, BB><<<grid, qk::kThreads, smem, st>>>(tq, tk, tv, p);                      \
   } while (0)
   if (mode == qk::kStats) {
     if (d.B == 128) MF_QK(qk::kStats, 128); else MF_QK(qk::kStats, 64);
@@ -446,14 +489,15 @@ static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, c
 cudaError_t launch_stats_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                             const void* Q, const void* K, float* lse, float* part,
                             cudaStream_t st) {
-  return launch_qk(qk::kStats, d, sz, m, Q, K, lse, part, nullptr, nullptr, st);
+  return launch_qk(qk::kStats, d, sz, m, Q, K, lse, part, nullptr, nullptr, 0, st);
 }
 
 cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                               const void* Q, const void* K, const float* lse,
-                              const int32_t* slot, void* values, cudaStream_t st) {
+                              const int32_t* slot, void* values, int64_t capacity,
+                              cudaStream_t st) {
   return launch_qk(qk::kExtract, d, sz, m, Q, K, const_cast<float*>(lse), nullptr, slot,
-                   values, st);
+                   values, capacity, st);
 }
 
 }  // namespace mf

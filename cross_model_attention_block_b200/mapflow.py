@@ -216,9 +216,9 @@ class Cache:
         return int(self.row_ptr[-1].item())
 
     def values_view(self):
-        """values as [capacity, B/16, B, Hs, 16] (stored order, see the C header)."""
+        """values as [capacity, Hs, B rows, B keys] (see the C header)."""
         B, Hs = self.ctx.B, self.ctx.Hs
-        return self.values[: self.capacity * B * B * Hs].view(self.capacity, B // 16, B, Hs, 16)
+        return self.values[: self.capacity * B * B * Hs].view(self.capacity, Hs, B, B)
 
 
 def select_extract(ctx: Context, Q, K, lse, mass, tau, cache: Cache | None = None):

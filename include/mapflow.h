@@ -84,10 +84,8 @@ typedef struct {
  *          global query block.
  *  values: kept probability blocks P_h[i,j] = exp(s_h[i,j] - lse_h[i]) for
  *          j <= i (0 above the diagonal and beyond the sequence end), of
- *          dtype dt, layout [nnz][B/16][B][Hs][16]: entry e, key group
- *          jg = j/16, row i, head h, key j%16 -- except that the two 8-key
- *          halves of the 16 keys are stored swapped when bit 2 of h is set
- *          (stored position (j%16) ^ (8 * ((h>>2)&1))).
+ *          dtype dt, layout [nnz][Hs][B][B]: entry e, head h, row i of the
+ *          query block, key j of the key block (head-major planes).
  *  cu_seqlens, nseq: the context the cache was built from (device). */
 typedef struct {
   int64_t nqb_total;

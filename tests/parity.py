@@ -123,11 +123,10 @@ def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
         # extracted probability blocks
         if check_values:
             for e, kb in zip(range(rp[g], rp[g + 1]), kept_g):
-                blk = f64(vals[e])                       # [B/16, B, Hs, 16] stored order
+                got = f64(vals[e])                       # [Hs, B rows, B keys]
                 ref = np.zeros((P.shape[0], B, B))
                 hi = min(P.shape[2], (kb + 1) * B)
                 ref[:, : i1 - i0, : hi - kb * B] = P[:, :, kb * B:hi]
-                got = unswizzle_block(blk, ctx.Hs, B)    # [Hs, B, B]
                 if dtype == torch.float32:
                     np.testing.assert_allclose(got, ref, rtol=2e-5, atol=1e-7)
                 else:
@@ -141,18 +140,6 @@ def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
         worst = max(worst, err)
         assert err <= tol, f"O seq {s} qb {qb}: rel err {err:.3e} > {tol}"
     return len(picks), n_ex, worst
-
-
-def unswizzle_block(blk, Hs, B):
-    """Stored [B/16, B, Hs, 16] (halves swapped for heads with bit 2 set) ->
-    logical [Hs, B rows, B keys]."""
-    out = np.empty((Hs, B, B))
-    for h in range(Hs):
-        sw = 8 if (h >> 2) & 1 else 0
-        idx = np.arange(16) ^ sw              # logical key -> stored slot
-        grp = blk[:, :, h, :][:, :, idx]      # [B/16, B, 16] logical keys
-        out[h] = np.transpose(grp, (1, 0, 2)).reshape(B, B)
-    return out
 
 
 def all_picks(ctx):

@@ -248,7 +248,10 @@ mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int3
   if (!status_word()) return fail(MF_ERR_CUDA, "no CUDA device");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (sz.nqb == 0) return MF_OK;
-  cudaError_t e = launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, s);
+  if (v->page_table && v->npages < 1) return fail(MF_ERR_INVALID_ARG, "npages < 1");
+  cudaError_t e = mapped_av_tc_supported(d, Hr, *v)
+                      ? launch_mapped_av_tc(*cache, d, sz, Hr, W, *v, O, s)
+                      : launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, s);
   if (e != cudaSuccess) return cuda_fail(e, "mapped av");
   return MF_OK;
 }

@@ -1,6 +1,7 @@
 // Internal host-side interface between the translation units of libmapflow.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -58,6 +59,16 @@ cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const Meta
                               const void* Q, const void* K, const float* lse,
                               const int32_t* slot, void* values, int64_t capacity,
                               cudaStream_t st);
+
+// Tensor map of a bf16 tensor (rank <= 5; strides of dims 1.. in bytes;
+// swizzle_bytes 0, 32, 64 or 128).
+cudaError_t make_tmap_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                           const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
+
+bool mapped_av_tc_supported(const mf_attn_desc& d, int Hr, const mf_v_desc& v);
+cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, const Sizes& sz,
+                                int Hr, const void* W, const mf_v_desc& v, void* O,
+                                cudaStream_t st);
 
 cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                               const void* Q, const void* K, float* lse, float* part,

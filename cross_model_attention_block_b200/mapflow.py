@@ -48,7 +48,8 @@ class CsrCache(C.Structure):
 
 class VDesc(C.Structure):
     _fields_ = [("V", C.c_void_p), ("page_table", C.c_void_p), ("page_size", C.c_int32),
-                ("max_pages_per_seq", C.c_int32), ("Hkv", C.c_int32), ("d", C.c_int32)]
+                ("max_pages_per_seq", C.c_int32), ("npages", C.c_int64), ("Hkv", C.c_int32),
+                ("d", C.c_int32)]
 
 
 class MapflowError(RuntimeError):
@@ -246,8 +247,9 @@ def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None
     if O is None:
         O = torch.empty((ctx.ntok, Hr, ctx.d), dtype=ctx.dtype, device=W.device)
     maxp = 0 if page_table is None else int(page_table.shape[1])
+    npages = 0 if page_table is None else int(V.shape[0])
     vd = VDesc(V.data_ptr(), 0 if page_table is None else page_table.data_ptr(),
-               page_size, maxp, Hkv, ctx.d)
+               page_size, maxp, npages, Hkv, ctx.d)
     cs = cache.struct()
     _check(L.mf_mapped_av(C.byref(cs), C.byref(d), int(Hr), _ptr(W), C.byref(vd), _ptr(O),
                           _stream()))

@@ -106,12 +106,15 @@ typedef struct {
  *  page_table == NULL: V is [ntok][Hkv][d] (packed like Q).
  *  otherwise V is a page pool [npages][page_size][Hkv][d] and
  *  page_table[s * max_pages_per_seq + p] is the pool page holding tokens
- *  p*page_size .. of sequence s.  page_size must be a multiple of 16. */
+ *  p*page_size .. of sequence s; the pool holds npages pages.  page_size
+ *  must be a multiple of 16.  Rows of a last page past its sequence's end
+ *  must hold finite values (they are multiplied by zero). */
 typedef struct {
   const void* V;
   const int32_t* page_table;
   int32_t page_size;
   int32_t max_pages_per_seq;
+  int64_t npages;           /* pages in the pool (paged only) */
   int32_t Hkv, d;
 } mf_v_desc;
 

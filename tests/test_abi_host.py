@@ -92,10 +92,10 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.mf_select_extract(C.byref(dsc), P(16), P(16), P(16), P(16), 0.9,
                                  C.byref(wrong_rows), P(256), ws, None) == mfb.MF_ERR_INVALID_ARG
     # mapped AV: Hr must be a multiple of Hkv; page size rule
-    v = mfb.VDesc(16, None, 16, 0, 3, 64)
+    v = mfb.VDesc(16, None, 16, 0, 0, 3, 64)
     assert lib.mf_mapped_av(C.byref(cache), C.byref(dsc), 4, P(16), C.byref(v), P(16),
                             None) == mfb.MF_ERR_INVALID_ARG
-    v = mfb.VDesc(16, 16, 8, 64, 2, 64)
+    v = mfb.VDesc(16, 16, 8, 64, 10, 2, 64)
     assert lib.mf_mapped_av(C.byref(cache), C.byref(dsc), 4, P(16), C.byref(v), P(16),
                             None) == mfb.MF_ERR_INVALID_ARG
 

@@ -165,3 +165,45 @@ def test_varlen_paged_workload_sampled():
     O_c = mfb.mapped_av(gpu[2], w.Hr, x.W.cuda(), x.V.cuda(), w.Hkv)
     mfb.sync_status()
     assert torch.equal(O_c, gpu[3])
+
+
+@pytest.mark.parametrize("case", [
+    dict(lengths=[300, 200], Hs=40, Hr=32, Hkv=8, B=64, tau=0.9),
+    dict(lengths=[390], Hs=40, Hr=32, Hkv=8, B=128, tau=0.9),
+    dict(lengths=[257, 31], Hs=32, Hr=16, Hkv=4, B=64, tau=0.8),
+    dict(lengths=[160], Hs=16, Hr=16, Hkv=8, B=128, tau=0.95),
+], ids=["hs40_b64", "hs40_b128", "hs32_g4_b64", "hs16_g2_b128"])
+def test_mapped_av_on_an_oracle_built_cache(case):
+    """The fused kernel alone: cache (CSR + probability blocks) written from the
+    oracle, O compared with the oracle's."""
+    from oracle import mapflow_oracle as orc
+    w, x = synth.small_case(case["lengths"], case["Hs"], case["Hr"], case["Hkv"], 128,
+                            case["B"], case["tau"])
+    res, O_ref = orc.run_layer(x.Q, x.K, x.V, x.W, w.lengths, w.Hkv, w.B, w.tau,
+                               w.band_bias, w.band_width, want_values=True)
+    ctx = _ctx_of(w)
+    cache = mfb.Cache(ctx)
+    rows, cols, vals = [0], [], []
+    g = 0
+    for s, r in enumerate(res):
+        for qb in sorted(r):
+            rec = r[qb]
+            for kb in rec["kept"]:
+                cols.append(int(kb))
+                blk = np.zeros((w.Hs, w.B, w.B))
+                v = rec["values"][int(kb)]
+                blk[:, : v.shape[1], :] = v
+                vals.append(blk)
+            rows.append(rows[-1] + len(rec["kept"]))
+            cache.qb_seq[g] = s
+            cache.qb_idx[g] = qb
+            g += 1
+    cache.row_ptr.copy_(torch.tensor(rows, dtype=torch.int64))
+    cache.col_idx[: len(cols)].copy_(torch.tensor(cols, dtype=torch.int32))
+    vv = cache.values_view()
+    vv[: len(vals)].copy_(torch.from_numpy(np.stack(vals)).to(torch.bfloat16))
+    O = mfb.mapped_av(cache, w.Hr, x.W.cuda(), x.V.cuda(), w.Hkv)
+    mfb.sync_status()
+    O = O.double().cpu().numpy()
+    err = np.abs(O - O_ref).max() / np.abs(O_ref).max()
+    assert err <= 2e-2, err

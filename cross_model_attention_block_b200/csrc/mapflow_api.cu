@@ -31,6 +31,8 @@ mf_status cuda_fail(cudaError_t e, const char* where) {
 }
 }  // namespace
 
+void set_last_error(const char* msg) { t_last_error = msg; }
+
 unsigned* status_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;

@@ -16,6 +16,9 @@ enum : unsigned { kStatusTimeout = 1u, kStatusCapacity = 2u };
 // Device address of the status word of the current device.
 unsigned* status_word();
 
+// Sets the text mf_last_error() returns to this thread.
+void set_last_error(const char* msg);
+
 // Per-context block layout, device arrays computed from cu_seqlens.
 struct Meta {
   int32_t* cu_qb;    // [nseq+1] prefix of ceil(L_s/B)

@@ -146,6 +146,27 @@ mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
                          float* lse, float* mass, void* ws, size_t ws_bytes,
                          mf_stream_t stream);
 
+/* Block statistics without a caller workspace.  The article has no
+ * counterpart: this exists for callers that cannot allocate device memory,
+ * such as a serving engine that gave all free HBM to its KV-cache pool, or a
+ * host program with a fixed memory plan and no device allocator.
+ *  Same inputs, outputs and results as mf_block_stats; the scratch comes from
+ *  one array the library keeps in device memory (8 MiB, held by every GPU that
+ *  loads the library until the process exits).  A context needing more than
+ *  mf_block_stats_noalloc_max_workspace() bytes (see
+ *  mf_block_stats_workspace) is rejected with MF_ERR_WORKSPACE and a message.
+ *  Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ *  The first call on a device looks up the array's device address
+ *  (cudaGetSymbolAddress) with that device current; make that first call
+ *  before any stream capture.
+ *  Every call shares the one array and leaves its contents behind; no part
+ *  of it needs to start at zero, since each call writes every scratch word it
+ *  reads.  Calls that overlap on the GPU (other streams, or other host
+ *  threads using the same device) race on the array: serialize them. */
+size_t mf_block_stats_noalloc_max_workspace(void);
+mf_status mf_block_stats_noalloc(const mf_attn_desc* desc, const void* Q, const void* K,
+                                 float* lse, float* mass, mf_stream_t stream);
+
 /* Stage 2, selection and extraction (article: keep the important blocks by
  * cumulative attention probability; extract only the kept blocks).
  * Per global query block: order key blocks by mass descending, ties to the

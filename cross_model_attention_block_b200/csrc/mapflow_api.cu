@@ -228,15 +228,14 @@ mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void*
   return MF_OK;
 }
 
-mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int32_t Hr,
-                       const void* W, const mf_v_desc* v, void* O, mf_stream_t stream) {
-  Sizes sz;
-  mf_status st = check_desc(desc, &sz);
+static mf_status check_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int32_t Hr,
+                          const mf_v_desc* v, Sizes* sz) {
+  mf_status st = check_desc(desc, sz);
   if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
-  st = check_cache(cache, d, sz);
+  st = check_cache(cache, d, *sz);
   if (st != MF_OK) return st;
-  if (!W || !v || !v->V || !O) return fail(MF_ERR_INVALID_ARG, "W, V or O is NULL");
+  if (!v || !v->V) return fail(MF_ERR_INVALID_ARG, "V is NULL");
   if (v->d != d.d) return fail(MF_ERR_INVALID_ARG, "V head dim differs from the descriptor");
   if (v->Hkv < 1 || Hr < 1 || Hr % v->Hkv != 0)
     return fail(MF_ERR_INVALID_ARG, "Hr must be a positive multiple of Hkv");
@@ -244,16 +243,45 @@ mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int3
   if (v->page_table) {
     if (v->page_size < 16 || v->page_size % 16 != 0)
       return fail(MF_ERR_INVALID_ARG, "page_size must be a positive multiple of 16");
-    if (int64_t(v->max_pages_per_seq) * v->page_size < sz.max_len)
+    if (int64_t(v->max_pages_per_seq) * v->page_size < sz->max_len)
       return fail(MF_ERR_INVALID_ARG, "max_pages_per_seq * page_size below a sequence length");
+    if (v->npages < 1) return fail(MF_ERR_INVALID_ARG, "npages < 1");
   }
+  return MF_OK;
+}
+
+// 16-key groups of a context: sum_s ceil(L_s / 16).
+static int64_t key_groups(const mf_attn_desc& d) {
+  int64_t g = 0;
+  for (int s = 0; s < d.nseq; ++s) g += (int64_t(d.cu_seqlens_host[s + 1]) - d.cu_seqlens_host[s] + 15) / 16;
+  return g;
+}
+
+size_t mf_mapped_av_workspace(const mf_csr_cache* cache, const mf_attn_desc* desc, int32_t Hr,
+                              const mf_v_desc* v) {
+  Sizes sz;
+  if (check_av(cache, desc, Hr, v, &sz) != MF_OK) return 0;
+  if (!mapped_av_tc_supported(*desc, Hr, *v)) return 256;
+  return mapped_av_tc_workspace(desc->nseq, key_groups(*desc), v->Hkv);
+}
+
+mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int32_t Hr,
+                       const void* W, const mf_v_desc* v, void* O, void* ws, size_t ws_bytes,
+                       mf_stream_t stream) {
+  Sizes sz;
+  mf_status st = check_av(cache, desc, Hr, v, &sz);
+  if (st != MF_OK) return st;
+  const mf_attn_desc& d = *desc;
+  if (!W || !O) return fail(MF_ERR_INVALID_ARG, "W or O is NULL");
+  const bool tc = mapped_av_tc_supported(d, Hr, *v);
+  if (tc && (!ws || !aligned256(ws) ||
+             ws_bytes < mapped_av_tc_workspace(d.nseq, key_groups(d), v->Hkv)))
+    return fail(MF_ERR_WORKSPACE, "workspace missing, not 256-byte aligned or too small");
   if (!status_word()) return fail(MF_ERR_CUDA, "no CUDA device");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (sz.nqb == 0) return MF_OK;
-  if (v->page_table && v->npages < 1) return fail(MF_ERR_INVALID_ARG, "npages < 1");
-  cudaError_t e = mapped_av_tc_supported(d, Hr, *v)
-                      ? launch_mapped_av_tc(*cache, d, sz, Hr, W, *v, O, s)
-                      : launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, s);
+  cudaError_t e = tc ? launch_mapped_av_tc(*cache, d, sz, Hr, W, *v, O, ws, key_groups(d), s)
+                     : launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, s);
   if (e != cudaSuccess) return cuda_fail(e, "mapped av");
   return MF_OK;
 }

@@ -29,10 +29,18 @@ __device__ __forceinline__ int upper_index(const I* a, int n, int64_t v) {
   return lo;
 }
 
-// Element offset of (entry e, head h, row i, key j) in the CSR value array
-// [nnz][Hs][B][B].
+// Element offset of (entry e, head h, row i, key j) in the CSR value array.
+// Layout [nnz][B/16 key groups][B/8 row slices][2 halves][Hs][64]: one
+// (entry, key group, row slice) -- 8 rows x 16 keys, all heads -- is one
+// contiguous stage of the fused kernel, stored exactly as the 128-byte-swizzled
+// MN-major operand of its head-mixing MMA: pair m = (i%8)*16 + j%16, half
+// m/64, and inside a 128-byte line (head h) the 16-byte chunk (m%64)/8 sits at
+// chunk ((m%64)/8) ^ (h%8).
 __device__ __forceinline__ int64_t value_offset(int64_t e, int i, int h, int j, int B, int Hs) {
-  return ((e * Hs + h) * B + i) * int64_t(B) + j;
+  const int64_t line = ((((e * (B >> 4) + (j >> 4)) * (B >> 3) + (i >> 3)) * 2 + ((i & 7) >> 2)) *
+                            Hs + h);
+  const int chunk = (((i & 3) << 1) | ((j >> 3) & 1)) ^ (h & 7);
+  return line * 64 + chunk * 8 + (j & 7);
 }
 
 __device__ __forceinline__ uint64_t global_ns() {

@@ -69,9 +69,12 @@ cudaError_t make_tmap_bf16(CUtensorMap* m, const void* base, int rank, const uin
                            const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
 
 bool mapped_av_tc_supported(const mf_attn_desc& d, int Hr, const mf_v_desc& v);
+// Workspace of the tensor-core fused kernel: per-sequence 16-key-group prefix
+// sums and V regrouped per 16 keys into operand images (4096 * Hkv bytes each).
+size_t mapped_av_tc_workspace(int nseq, int64_t key_groups, int Hkv);
 cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, const Sizes& sz,
-                                int Hr, const void* W, const mf_v_desc& v, void* O,
-                                cudaStream_t st);
+                                int Hr, const void* W, const mf_v_desc& v, void* O, void* ws,
+                                int64_t key_groups, cudaStream_t st);
 
 cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                               const void* Q, const void* K, float* lse, float* part,

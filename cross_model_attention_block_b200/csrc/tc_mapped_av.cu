@@ -1,4 +1,4 @@
-// Fused map-mix x V on B200 (bf16, d = 128).
+// Fused map-mix x V on B200 (bf16, d = 128), both products on tcgen05.
 //
 // MapFlow article (163.com, section on the three system components, third
 // component): the fused kernel reads the kept sparse blocks, forms the linear
@@ -8,20 +8,27 @@
 //
 //   O_r[i,:] = sum_{kb kept} sum_{j in kb} (sum_h W[r,h] P_h[i,j]) V_{g(r)}[j,:]
 //
-// One CTA owns a 16-row slice of one query block and all Hr receiver heads, so
-// every map byte is read from HBM once.  The kept key blocks are walked in
-// stages of 16 keys:
-//  * warp 0 (one thread) TMA-loads the map slab [16 rows][Hs][16 keys] with one
-//    4-D box (hardware 32-byte swizzle) and V [16 keys][Hkv][128] with one 3-D
-//    box (128-byte swizzle; with paged V the 16 keys are one page);
-//  * warps 4..7 mix: mma.sync m16n8k16 with the map slab as A (keys x heads,
-//    loaded transposed by ldmatrix) and W^T held in registers as B, giving the
-//    mixed map M (16 keys x Hr heads per row), written as bf16 into the
-//    MN-major B operand of the next product;
-//  * warp 1 (one thread) issues, per GQA group g, one tcgen05.mma
-//    O^T_g[128 x 16G] += V_g^T[128 x 16] M^T_g[16 x 16G] (M = d = 128, N = 16
-//    rows x G heads), with O^T for all groups resident in the 512 TMEM columns;
-//  * at the end warps 4..7 read O^T from TMEM (lane = d) and store O.
+// One CTA owns an 8-row slice of one query block and all Hr receiver heads,
+// so every map byte is read from HBM once.  Kept key blocks are walked in
+// stages of 16 keys; a stage moves two contiguous chunks with plain bulk
+// copies: the map slab (8 rows x 16 keys x Hs heads, stored by the cache in
+// exactly the operand layout of the mixing MMA) and the V image of those 16
+// keys (prepared once per call by k_v_format).  Per stage:
+//   1. mix MMA   Mix[128 pairs x Hr] = Map[128 pairs x Hs] . W^T[Hs x Hr]
+//      (tcgen05, M = 128 (row, key) pairs, K = Hs padded to a multiple of 16
+//      with zero W rows; two accumulators in TMEM);
+//   2. convert   four warps read Mix from TMEM, round to bf16 and store it as
+//      M^T_g[16 keys x 8 rows * G heads], the MN-major operand of step 3;
+//   3. O MMAs    O^T_g[128 d x 8G] += V_g^T[128 x 16] . M^T_g[16 x 8G] for every
+//      GQA group g (O^T of all groups resident in TMEM for the whole CTA).
+// The four converting warps also drive the tensor core: one of their lanes
+// issues mix(n+1) before stage n is converted and O(n) right after a named
+// barrier closes the conversion, so no stage waits on a hand-off to another
+// warp (an mbarrier round trip costs more than a stage's work).
+//
+// Why not mma.sync for the mix: on this part a legacy mma.sync takes a few
+// thousand cycles from issue to result unless hundreds are in flight; with
+// one stage's worth of work per warp that serialised the whole pipeline.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -34,12 +41,13 @@ using namespace sm100;
 
 namespace av {
 
-constexpr int kRows = 16;      // query rows per CTA
-constexpr int kKeys = 16;      // keys per stage (= MMA K)
+constexpr int kRows = 8;   // query rows per CTA
+constexpr int kKeys = 16;  // keys per stage
 constexpr int kD = 128;
-constexpr int kMaxStages = 3;
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxMapStages = 8;
+constexpr int kMixBufs = 2;  // mix accumulators in TMEM (mix(n+1) runs while n converts)
 
 struct Params {
   const int64_t* row_ptr;
@@ -47,62 +55,42 @@ struct Params {
   const int32_t* qb_seq;
   const int32_t* qb_idx;
   const int32_t* cu_seqlens;
-  const int32_t* page_table;  // NULL: contiguous V
+  const int32_t* cu_g;        // [nseq+1] prefix of ceil(L_s / 16)
+  const uint8_t* vimg;        // [groups][4096 * Hkv] V operand images
+  const __nv_bfloat16* values;
   const __nv_bfloat16* W;     // [Hr][Hs]
   __nv_bfloat16* O;           // [ntok][Hr][d]
   int64_t capacity;
   int64_t nqb;
-  int Hs, Hr, Hkv, G, B;
-  int page_size, max_pages;
-  // shared-memory layout (bytes from the 1024-aligned base)
-  uint32_t off_v, off_map, off_mt, v_bytes, map_bytes, mt_bytes, mt_group_stride;
-  uint32_t off_bar;
-  int stages;  // pipeline depth (2 or 3, whatever fits in shared memory)
+  int Hs, Hs_pad, Hr, Hkv, G, B;
+  uint32_t map_bytes;       // Hs * 256 (one stage)
+  uint32_t map_slot;        // map_bytes + 1 KB zero guard, 1 KB aligned
+  uint32_t v_bytes, mt_group_stride, mt_bytes, w_bytes;
+  uint32_t off_v, off_map, off_mt, off_w, off_bar;
+  int map_stages, vm_stages;
   unsigned* status;
 };
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& a0, uint32_t& a1, uint32_t& a2,
-                                          uint32_t& a3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& a0, uint32_t& a1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-               : "=r"(a0), "=r"(a1)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mma1688(float* c, uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(b0));
-}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Address of 16-byte chunk c (keys 8c..8c+7) of line (row i, head h) in the
-// map slab: lines of 32 bytes, 32-byte swizzle (chunk bit flips on line bit 2).
-__device__ __forceinline__ uint32_t map_addr(uint32_t base, int line, int c) {
-  return base + line * 32 + ((c ^ ((line >> 2) & 1)) << 4);
+// AND of a predicate over the 128 worker threads (named barrier 1).
+__device__ __forceinline__ bool epilogue_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v))
+      : "memory");
+  return r != 0;
 }
 
-// Stage walk: (entry e, key group kg) pairs of this query block, skipping key
+// Stage walk: (entry e, key group kg) pairs of one query block, skipping key
 // groups that start past the sequence end.
 struct Walk {
   int64_t e, e1;
@@ -115,10 +103,10 @@ struct Walk {
       ++e;
       if (e >= e1) return false;
       kb = col_idx[e];
-      int rem = L - kb * B;
+      const int rem = L - kb * B;
       nkg = (min(rem, B) + kKeys - 1) / kKeys;
       kg = -1;
-      if (nkg <= 0) { nkg = 0; continue; }
+      if (nkg <= 0) nkg = 0;
     }
   }
 };
@@ -136,17 +124,21 @@ __device__ __forceinline__ Walk make_walk(const Params& p, int64_t gqb, int L) {
   return w;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    k_mapped_av(const __grid_constant__ CUtensorMap tmMap, const __grid_constant__ CUtensorMap tmV,
-                const Params p) {
+template <int HR, int G>
+__global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
+  constexpr int HKV = HR / G;
+  constexpr int NO = kRows * G;          // O MMA N per group
+  constexpr uint32_t kMixCol = 8u * HR;  // first TMEM column of the mix accumulators
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const int kStages = p.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + p.off_bar);  // [stages]
-  uint64_t* mt_ready = full + kStages;                              // [stages]
-  uint64_t* done = mt_ready + kStages;                              // [stages]
-  uint64_t* final_bar = done + kStages;
+  const int MS = p.map_stages, VS = p.vm_stages;
+  uint64_t* map_full = reinterpret_cast<uint64_t*>(base + p.off_bar);  // [MS]
+  uint64_t* map_empty = map_full + MS;                                  // [MS]
+  uint64_t* v_full = map_empty + MS;                                    // [VS]
+  uint64_t* vm_empty = v_full + VS;                                     // [VS]
+  uint64_t* mix_full = vm_empty + VS;                                   // [kMixBufs]
+  uint64_t* final_bar = mix_full + kMixBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -160,13 +152,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (i0 >= L) return;                      // the whole slice is past the sequence end
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&mt_ready[i], 4);
-      mbar_init(&done[i], 1);
+    for (int i = 0; i < MS; ++i) {
+      mbar_init(&map_full[i], 1);
+      mbar_init(&map_empty[i], 1);
     }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&vm_empty[i], 1);
+    }
+    for (int i = 0; i < kMixBufs; ++i) mbar_init(&mix_full[i], 1);
     mbar_init(final_bar, 1);
     fence_barrier_init();
+  }
+  // W^T as the K-major operand [Hr rows][Hs_pad], core matrices of 8 rows x 16
+  // bytes, K chunks 128 bytes apart, row groups Hs_pad * 16 bytes apart; zero
+  // past Hs.  The 1 KB guard after every map slot is zeroed (the padded K
+  // step of the mix reads it).
+  {
+    uint8_t* wt = base + p.off_w;
+    for (int idx = threadIdx.x; idx < HR * p.Hs_pad; idx += kThreads) {
+      const int r = idx / p.Hs_pad, h = idx % p.Hs_pad;
+      const __nv_bfloat16 w = h < p.Hs ? p.W[r * p.Hs + h] : __float2bfloat16_rn(0.f);
+      *reinterpret_cast<__nv_bfloat16*>(wt + (r >> 3) * (p.Hs_pad * 16) + (h >> 3) * 128 +
+                                        (r & 7) * 16 + (h & 7) * 2) = w;
+    }
+    for (int st = 0; st < MS; ++st) {
+      uint32_t* g = reinterpret_cast<uint32_t*>(base + p.off_map + st * p.map_slot + p.map_bytes);
+      for (int k = threadIdx.x; k < 256; k += kThreads) g[k] = 0u;
+    }
+    fence_proxy_async_smem();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -174,177 +188,145 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(base);
-  const int N = kRows * p.G;  // MMA N per group
+  const int S16 = p.B / 16, S8 = p.B / 8;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------- map producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmMap);
-      tma_prefetch_desc(&tmV);
       Walk wk = make_walk(p, gqb, L);
       int n = 0;
       while (wk.next()) {
-        const int st = n % kStages;
-        if (!mbar_wait(&done[st], ((n / kStages) & 1) ^ 1, p.status)) break;
-        // exact bytes of the two boxes: 16 keys x Hs x 16 rows, 16 keys x Hkv x 128
-        mbar_expect_tx(&full[st], uint32_t(512 * p.Hs) + uint32_t(4096 * p.Hkv));
-        // map slab: keys 16kg.., all heads, rows 16*slice.., entry e
-        asm volatile(
-            "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-            " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(sbase + p.off_map + st * p.map_bytes),
-            "l"(reinterpret_cast<uint64_t>(&tmMap)), "r"(smem_u32(&full[st])),
-            "r"(wk.kg * kKeys), "r"(0), "r"(slice * kRows), "r"(int32_t(wk.e))
-            : "memory");
-        // V rows of these 16 keys
-        const int j = wk.kb * p.B + wk.kg * kKeys;  // key (in the sequence)
-        int row;
-        if (p.page_table) {
-          const int page = p.page_table[int64_t(s) * p.max_pages + j / p.page_size];
-          row = page * p.page_size + (j % p.page_size);
-        } else {
-          row = seq0 + j;
-        }
-        tma_load_3d(base + p.off_v + st * p.v_bytes, &tmV, &full[st], 0, row, 0);
+        const int st = n % MS;
+        if (!mbar_wait(&map_empty[st], ((n / MS) & 1) ^ 1, p.status)) break;
+        mbar_expect_tx(&map_full[st], p.map_bytes);
+        const int64_t line0 = ((wk.e * S16 + wk.kg) * S8 + slice) * 2 * p.Hs;
+        bulk_load(base + p.off_map + st * p.map_slot, p.values + line0 * 64, p.map_bytes,
+                  &map_full[st]);
         ++n;
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 2) {
+    // --------------------------------------------------------- V producer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, N, 1, 1);
       Walk wk = make_walk(p, gqb, L);
+      const int64_t g0 = p.cu_g[s];
       int n = 0;
       while (wk.next()) {
-        const int st = n % kStages;
-        const uint32_t ph = (n / kStages) & 1;
-        if (!mbar_wait(&full[st], ph, p.status)) break;
-        if (!mbar_wait(&mt_ready[st], ph, p.status)) break;
+        const int st = n % VS;
+        if (!mbar_wait(&vm_empty[st], ((n / VS) & 1) ^ 1, p.status)) break;
+        mbar_expect_tx(&v_full[st], p.v_bytes);
+        const int64_t grp = g0 + (wk.kb * p.B + wk.kg * kKeys) / kKeys;
+        bulk_load(base + p.off_v + st * p.v_bytes, p.vimg + grp * p.v_bytes, p.v_bytes,
+                  &v_full[st]);
+        ++n;
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ workers
+    // One lane issues every MMA; all 128 threads (one per mix-accumulator
+    // lane = (row, key) pair) convert.  mix(n+1) is issued before stage n is
+    // converted, so its tensor-core time overlaps the conversion.
+    const int q = warp & 3;  // TMEM lane quarter: pairs 32q .. 32q+31
+    const int m = q * 32 + lane;
+    const int r8 = m >> 4, k16 = m & 15;
+    const bool leader = threadIdx.x == 128;
+    const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
+    const uint32_t idesc_mix = idesc_bf16(128, HR, 1, 0);  // A MN-major, B K-major
+    const uint32_t idesc_o = idesc_bf16(128, NO, 1, 1);    // A, B MN-major
+    const int ksteps = p.Hs_pad / 16;
+    // mix(n): Mix[pairs x Hr] = Map[pairs x Hs] . W^T into accumulator n % kMixBufs
+    auto issue_mix = [&](int n) -> bool {
+      const int ms = n % MS;
+      if (!mbar_wait(&map_full[ms], (n / MS) & 1, p.status)) return false;
+      tc_fence_after();
+      const uint32_t ma = sbase + p.off_map + ms * p.map_slot;
+      for (int kk = 0; kk < ksteps; ++kk) {
+        // A = map slab: MN-major, 128-byte swizzle, pair halves Hs * 128 B apart,
+        // 8-head groups 1 KB apart; B = W^T: K-major, no swizzle
+        const uint64_t adesc = smem_desc(ma + kk * 2048, p.Hs * 128, 1024, kSwizzle128);
+        const uint64_t bdesc =
+            smem_desc(sbase + p.off_w + kk * 256, 128, p.Hs_pad * 16, kSwizzleNone);
+        mma_bf16_ss(tmem + kMixCol + (n % kMixBufs) * HR, adesc, bdesc, idesc_mix, kk > 0);
+      }
+      mma_commit(&map_empty[ms]);
+      mma_commit(&mix_full[n % kMixBufs]);
+      return true;
+    };
+    Walk wk = make_walk(p, gqb, L);
+    Walk ahead = wk;
+    bool more = ahead.next();  // `ahead` runs one stage in front of `wk`
+    bool lead_ok = true;
+    if (leader && more) lead_ok = issue_mix(0);
+    int n = 0;
+    while (wk.next()) {
+      more = ahead.next();
+      if (leader && more && lead_ok) lead_ok = issue_mix(n + 1);
+      const int db = n % kMixBufs, vs = n % VS;
+      bool ok = mbar_wait(&mix_full[db], (n / kMixBufs) & 1, p.status);
+      tc_fence_after();
+      float v[HR];
+      if constexpr (HR == 32) {
+        tmem_ld32(lane_addr + kMixCol + db * HR, v);
+      } else {
+        tmem_ld16(lane_addr + kMixCol + db * HR, v);
+      }
+      tmem_wait_ld();
+      ok = ok && mbar_wait(&vm_empty[vs], ((n / VS) & 1) ^ 1, p.status);  // M^T slot free
+      const int kvalid = min(kKeys, L - (wk.kb * p.B + wk.kg * kKeys));  // keys < L
+      const float z = (k16 < kvalid && i0 + r8 < L) ? 1.f : 0.f;
+      uint8_t* mt = base + p.off_mt + vs * p.mt_bytes + (k16 >> 3) * 128 + (k16 & 7) * 16;
+#pragma unroll
+      for (int r = 0; r < HR; r += 2) {
+        const int g = r / G, rl = r % G;
+        const int nn = r8 * G + rl;  // MMA N index of (row r8, head r)
+        *reinterpret_cast<uint32_t*>(mt + g * p.mt_group_stride + (nn >> 3) * 256 +
+                                     ((nn & 7) << 1)) = pack_bf16(v[r] * z, v[r + 1] * z);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      // all four warps' M^T (and their reads of accumulator db) are done
+      if (!epilogue_all(ok)) break;
+      if (leader) {
+        // O(n): O^T_g += V_g^T . M^T_g for every GQA group
+        if (!mbar_wait(&v_full[vs], (n / VS) & 1, p.status)) lead_ok = false;
         tc_fence_after();
-        const uint32_t va = sbase + p.off_v + st * p.v_bytes;
-        const uint32_t mb = sbase + p.off_mt + st * p.mt_bytes;
-        for (int g = 0; g < p.Hkv; ++g) {
+        const uint32_t va = sbase + p.off_v + vs * p.v_bytes;
+        const uint32_t mb = sbase + p.off_mt + vs * p.mt_bytes;
+#pragma unroll
+        for (int g = 0; g < HKV; ++g) {
           // A = V_g^T: MN-major, 128-byte swizzle, d halves 2 KB apart, 8-key groups 1 KB apart
           const uint64_t adesc = smem_desc(va + g * 4096, 2048, 1024, kSwizzle128);
           // B = M^T_g: MN-major, no swizzle, n-chunks 256 B apart, 8-key groups 128 B apart
           const uint64_t bdesc = smem_desc(mb + g * p.mt_group_stride, 128, 256, kSwizzleNone);
-          mma_bf16_ss(tmem + g * N, adesc, bdesc, idesc, n > 0);
+          if (lead_ok) mma_bf16_ss(tmem + g * NO, adesc, bdesc, idesc_o, n > 0);
         }
-        mma_commit(&done[st]);
-        ++n;
+        mma_commit(&vm_empty[vs]);
       }
-      mma_commit(final_bar);
-    }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ mix warps
-    const int mw = warp - 4;  // rows 4mw .. 4mw+3 of the slice
-    const int nks16 = p.Hs / 16;
-    const bool has8 = (p.Hs & 15) != 0;
-    const int ntile = p.Hr / 8;
-    // W^T fragments (B operand): B[k = h][n = r], thread: n = lane/4, k = 2(lane%4)+{0,1}(+8)
-    uint32_t wb[4][5][2];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int ks = 0; ks < 5; ++ks)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int r = nt * 8 + lane / 4;
-          const int h = ks * 16 + hh * 8 + 2 * (lane % 4);
-          float w0 = 0.f, w1 = 0.f;
-          if (nt < ntile && h < p.Hs) {
-            w0 = __bfloat162float(p.W[r * p.Hs + h]);
-            w1 = __bfloat162float(p.W[r * p.Hs + h + 1]);
-          }
-          wb[nt][ks][hh] = pack_bf16(w0, w1);
-        }
-    Walk wk = make_walk(p, gqb, L);
-    int n = 0;
-    while (wk.next()) {
-      const int st = n % kStages;
-      const uint32_t ph = (n / kStages) & 1;
-      if (!mbar_wait(&full[st], ph, p.status)) break;
-      const uint32_t mp = sbase + p.off_map + st * p.map_bytes;
-      uint8_t* mt = base + p.off_mt + st * p.mt_bytes;
-      const int kvalid = min(kKeys, L - (wk.kb * p.B + wk.kg * kKeys));  // keys < L
-#pragma unroll 1
-      for (int ii = 0; ii < 4; ++ii) {
-        const int i = mw * 4 + ii;  // row in the slice
-        float acc[4][4];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc[nt][k] = 0.f;
-        // ldmatrix rows: lanes 0-7 heads h0+l keys 0-7, 8-15 heads h0+l keys 8-15,
-        // 16-23 heads h0+8+l keys 0-7, 24-31 heads h0+8+l keys 8-15
-        const int lh = (lane & 7) + ((lane >> 4) << 3);
-        const int lc = (lane >> 3) & 1;
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          if (ks < nks16) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(map_addr(mp, i * p.Hs + ks * 16 + lh, lc), a0, a1, a2, a3);
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-              if (nt < ntile) mma16816(acc[nt], a0, a1, a2, a3, wb[nt][ks][0], wb[nt][ks][1]);
-          }
-        }
-        if (has8) {
-          uint32_t a0, a1;
-          ldsm_x2_t(map_addr(mp, i * p.Hs + nks16 * 16 + (lane & 7), (lane >> 3) & 1), a0, a1);
-#pragma unroll
-          for (int nt = 0; nt < 4; ++nt)
-            if (nt < ntile) {
-              // the k8 step uses the first register of the last 16-head fragment slot
-              uint32_t b = (nks16 == 0) ? wb[nt][0][0]
-                         : (nks16 == 1) ? wb[nt][1][0]
-                         : (nks16 == 2) ? wb[nt][2][0]
-                         : (nks16 == 3) ? wb[nt][3][0] : wb[nt][4][0];
-              mma1688(acc[nt], a0, a1, b);
-            }
-        }
-        // D fragment: keys j = lane/4 (+8), heads r = 8nt + 2(lane%4) + {0,1}
-        const int j0 = lane >> 2;
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          if (nt >= ntile) continue;
-          const int r = nt * 8 + 2 * (lane & 3);
-          const int g = r / p.G, rl = r % p.G;
-          const int nn = i * p.G + rl;  // MMA N index of (row i, head r)
-          uint8_t* gb = mt + g * p.mt_group_stride + (nn >> 3) * 256 + ((nn & 7) << 1);
-          const float z0 = j0 < kvalid ? 1.f : 0.f, z1 = j0 + 8 < kvalid ? 1.f : 0.f;
-          *reinterpret_cast<uint32_t*>(gb + (j0 >> 3) * 128 + (j0 & 7) * 16) =
-              pack_bf16(acc[nt][0] * z0, acc[nt][1] * z0);
-          *reinterpret_cast<uint32_t*>(gb + ((j0 + 8) >> 3) * 128 + ((j0 + 8) & 7) * 16) =
-              pack_bf16(acc[nt][2] * z1, acc[nt][3] * z1);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&mt_ready[st]);
       ++n;
     }
+    if (leader) mma_commit(final_bar);
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;
-    const int c = quarter * 32 + lane;  // d index = TMEM lane
-    bool ok = mbar_wait(final_bar, 0, p.status);
+    const int c = q * 32 + lane;  // d index = TMEM lane
+    const bool ok = mbar_wait(final_bar, 0, p.status);
     tc_fence_after();
-    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
-    for (int g = 0; g < p.Hkv; ++g) {
-      for (int c0 = 0; c0 < N; c0 += 32) {
-        float v[32];
-        tmem_ld32(lane_addr + g * N + c0, v);
+#pragma unroll 1
+    for (int g = 0; g < HKV; ++g) {
+#pragma unroll
+      for (int c0 = 0; c0 < NO; c0 += 16) {
+        float o[16];
+        tmem_ld16(lane_addr + g * NO + c0, o);
         tmem_wait_ld();
         if (!ok || n == 0) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = 0.f;
+          for (int k = 0; k < 16; ++k) o[k] = 0.f;
         }
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
+        for (int k = 0; k < 16; ++k) {
           const int nn = c0 + k;
-          const int i = nn / p.G, rl = nn % p.G;
+          const int i = nn / G, rl = nn % G;
           const int row = i0 + i;
           if (row < L)
-            p.O[(int64_t(seq0 + row) * p.Hr + g * p.G + rl) * kD + c] = __float2bfloat16_rn(v[k]);
+            p.O[(int64_t(seq0 + row) * HR + g * G + rl) * kD + c] = __float2bfloat16_rn(o[k]);
         }
       }
     }
@@ -355,6 +337,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// Prefix sums of 16-key groups per sequence.
+__global__ void k_group_meta(int nseq, const int32_t* __restrict__ cu_seqlens, int32_t* cu_g) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int32_t g = 0;
+  cu_g[0] = 0;
+  for (int s = 0; s < nseq; ++s) {
+    g += (cu_seqlens[s + 1] - cu_seqlens[s] + 15) / 16;
+    cu_g[s + 1] = g;
+  }
+}
+
+// V regrouped per (sequence, 16-key group) into the image the O MMA reads as
+// its A operand: chunk (group g, d half) of 16 keys x 64 d, rows of 128 bytes,
+// 16-byte chunk index XOR key % 8 (128-byte swizzle).  Keys past the sequence
+// end are zero.  One CTA per image.
+__global__ void __launch_bounds__(256) k_v_format(
+    const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ page_table, int page_size,
+    int max_pages, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ cu_g,
+    int nseq, int Hkv, uint8_t* __restrict__ out) {
+  const int64_t grp = blockIdx.x;
+  const int s = upper_index(cu_g, nseq, grp);
+  const int kg = int(grp - cu_g[s]);
+  const int seq0 = cu_seqlens[s];
+  const int L = cu_seqlens[s + 1] - seq0;
+  const int chunks_per_key = Hkv * 16;  // 16-byte chunks of one key row (Hkv x 128 x 2 B)
+  const uint32_t img = 4096u * uint32_t(Hkv);
+  uint8_t* dst = out + grp * int64_t(img);
+  for (int q = threadIdx.x; q < kKeys * chunks_per_key; q += blockDim.x) {
+    const int k = q / chunks_per_key, cc = q % chunks_per_key;
+    const int j = kg * kKeys + k;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (j < L) {
+      int64_t row;
+      if (page_table) {
+        const int page = page_table[int64_t(s) * max_pages + j / page_size];
+        row = int64_t(page) * page_size + (j % page_size);
+      } else {
+        row = seq0 + j;
+      }
+      val = reinterpret_cast<const uint4*>(V + row * int64_t(Hkv) * kD)[cc];
+    }
+    const int g = cc >> 4, dch = cc & 15;  // group, 16-byte chunk of the 128 d
+    const int half = dch >> 3, c8 = dch & 7;
+    const uint32_t o = uint32_t((2 * g + half) * 2048 + k * 128 + ((c8 ^ (k & 7)) << 4));
+    *reinterpret_cast<uint4*>(dst + o) = val;
+  }
+}
+
 }  // namespace av
 
 // ------------------------------------------------------------------- host side
@@ -362,74 +392,92 @@ __global__ void __launch_bounds__(kThreads, 1)
 bool mapped_av_tc_supported(const mf_attn_desc& d, int Hr, const mf_v_desc& v) {
   if (d.dt != MF_BF16 || d.d != 128 || v.d != 128) return false;
   if (d.Hs % 8 != 0 || d.Hs > 64) return false;
-  if (Hr > 32 || Hr % 8 != 0 || v.Hkv < 1 || Hr % v.Hkv != 0) return false;
+  if ((Hr != 16 && Hr != 32) || v.Hkv < 1 || Hr % v.Hkv != 0) return false;
   const int G = Hr / v.Hkv;
   return G == 2 || G == 4 || G == 8;
 }
 
+size_t mapped_av_tc_workspace(int nseq, int64_t key_groups, int Hkv) {
+  const size_t meta = (size_t(nseq + 1) * 4 + 255) & ~size_t(255);
+  return meta + size_t(key_groups) * 4096u * size_t(Hkv) + 1024;
+}
+
 cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, const Sizes& sz,
-                                int Hr, const void* W, const mf_v_desc& v, void* O,
-                                cudaStream_t st) {
-  if (c.nnz_capacity < 1 || sz.nqb == 0) return cudaSuccess;
+                                int Hr, const void* W, const mf_v_desc& v, void* O, void* ws,
+                                int64_t key_groups, cudaStream_t st) {
+  if (c.nnz_capacity < 1 || sz.nqb == 0 || key_groups == 0) return cudaSuccess;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  int32_t* cu_g = reinterpret_cast<int32_t*>(wsb);
+  const size_t meta = (size_t(d.nseq + 1) * 4 + 255) & ~size_t(255);
+  uint8_t* vimg = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(wsb + meta) + 1023) &
+                                             ~uintptr_t(1023));
+  av::k_group_meta<<<1, 32, 0, st>>>(d.nseq, d.cu_seqlens, cu_g);
+  av::k_v_format<<<unsigned(key_groups), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(v.V), v.page_table, v.page_table ? v.page_size : 16,
+      v.max_pages_per_seq, d.cu_seqlens, cu_g, d.nseq, v.Hkv, vimg);
+
   av::Params p{};
   p.row_ptr = c.row_ptr;
   p.col_idx = c.col_idx;
   p.qb_seq = c.qb_seq;
   p.qb_idx = c.qb_idx;
   p.cu_seqlens = d.cu_seqlens;
-  p.page_table = v.page_table;
+  p.cu_g = cu_g;
+  p.vimg = vimg;
+  p.values = static_cast<const __nv_bfloat16*>(c.values);
   p.W = static_cast<const __nv_bfloat16*>(W);
   p.O = static_cast<__nv_bfloat16*>(O);
   p.capacity = c.nnz_capacity;
   p.nqb = sz.nqb;
   p.Hs = d.Hs;
+  p.Hs_pad = (d.Hs + 15) / 16 * 16;
   p.Hr = Hr;
   p.Hkv = v.Hkv;
   p.G = Hr / v.Hkv;
   p.B = d.B;
-  p.page_size = v.page_table ? v.page_size : 16;
-  p.max_pages = v.max_pages_per_seq;
   p.status = status_word();
-  // shared memory: V stages (1024-aligned), map stages, mixed-map stages, barriers
+  p.map_bytes = 256u * uint32_t(d.Hs);
+  p.map_slot = (p.map_bytes + 1024u + 1023u) & ~1023u;
   p.v_bytes = 4096u * uint32_t(v.Hkv);
-  p.map_bytes = ((512u * uint32_t(d.Hs)) + 1023u) & ~1023u;
-  p.mt_group_stride = 512u * uint32_t(p.G) + 16u;
+  p.mt_group_stride = 256u * uint32_t(p.G) + 16u;
   p.mt_bytes = (uint32_t(v.Hkv) * p.mt_group_stride + 127u) & ~127u;
-  const uint32_t per_stage = p.v_bytes + p.map_bytes + p.mt_bytes;
-  int nst = 3;
-  if (size_t(nst) * per_stage + 2048 > 227u * 1024u) nst = 2;
-  p.stages = nst;
+  p.w_bytes = (uint32_t(Hr) * uint32_t(p.Hs_pad) * 2u + 127u) & ~127u;
+  // deepest map ring that fits next to a V / mixed-map ring of 4 (else 3, 2)
+  const size_t budget = 227u * 1024u - 1024u - 512u - p.w_bytes;
+  int ms = 0, vs = 0;
+  for (int cand_vs = 4; cand_vs >= 2 && ms == 0; --cand_vs) {
+    const size_t fixed = size_t(cand_vs) * (p.v_bytes + p.mt_bytes);
+    for (int cand_ms = av::kMaxMapStages; cand_ms >= 2; --cand_ms)
+      if (fixed + size_t(cand_ms) * p.map_slot <= budget) {
+        ms = cand_ms;
+        vs = cand_vs;
+        break;
+      }
+  }
+  if (ms == 0) return cudaErrorInvalidConfiguration;
+  p.map_stages = ms;
+  p.vm_stages = vs;
   p.off_v = 0;
-  p.off_map = nst * p.v_bytes;
-  p.off_mt = p.off_map + nst * p.map_bytes;
-  p.off_bar = (p.off_mt + nst * p.mt_bytes + 7u) & ~7u;
-  const size_t smem = size_t(p.off_bar) + (3 * nst + 1) * 8 + 16 + 1024;
-  if (smem > 227u * 1024u) return cudaErrorInvalidConfiguration;
-
-  CUtensorMap tmap, tv;
-  {
-    // values [cap][Hs][B][B] viewed as (key j, head h, row i, entry e)
-    const uint64_t B = uint64_t(d.B);
-    const uint64_t dims[4] = {B, uint64_t(d.Hs), B, uint64_t(c.nnz_capacity)};
-    const uint64_t strides[3] = {B * B * 2, B * 2, uint64_t(d.Hs) * B * B * 2};
-    const uint32_t box[4] = {16, uint32_t(d.Hs), 16, 1};
-    cudaError_t e = make_tmap_bf16(&tmap, c.values, 4, dims, strides, box, 32);
-    if (e != cudaSuccess) return e;
-  }
-  {
-    // V rows (tokens or pool rows) viewed as (d half, row, (group, half) chunk)
-    const uint64_t rows = v.page_table ? uint64_t(v.npages) * v.page_size : uint64_t(sz.ntok);
-    const uint64_t dims[3] = {64, rows, uint64_t(2 * v.Hkv)};
-    const uint64_t strides[2] = {uint64_t(v.Hkv) * 128 * 2, 128};
-    const uint32_t box[3] = {64, 16, uint32_t(2 * v.Hkv)};
-    cudaError_t e = make_tmap_bf16(&tv, v.V, 3, dims, strides, box, 128);
-    if (e != cudaSuccess) return e;
-  }
-  cudaError_t e = cudaFuncSetAttribute(av::k_mapped_av,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
+  p.off_map = vs * p.v_bytes;
+  p.off_mt = p.off_map + ms * p.map_slot;
+  p.off_w = p.off_mt + vs * p.mt_bytes;
+  p.off_bar = (p.off_w + p.w_bytes + 7u) & ~7u;
+  const size_t smem = size_t(p.off_bar) + (2 * ms + 2 * vs + av::kMixBufs + 1) * 8 + 16 + 1024;
   const unsigned grid = unsigned(sz.nqb) * unsigned(d.B / av::kRows);
-  av::k_mapped_av<<<grid, av::kThreads, smem, st>>>(tmap, tv, p);
+  cudaError_t e = cudaSuccess;
+#define MF_AV(HR, G)                                                                        \
+  do {                                                                                      \
+    e = cudaFuncSetAttribute(av::k_mapped_av<HR, G>,                                        \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));       \
+    if (e != cudaSuccess) return e;                                                         \
+    av::k_mapped_av<HR, G><<<grid, av::kThreads, smem, st>>>(p);                            \
+  } while (0)
+  if (Hr == 32) {
+    if (p.G == 2) MF_AV(32, 2); else if (p.G == 4) MF_AV(32, 4); else MF_AV(32, 8);
+  } else {
+    if (p.G == 2) MF_AV(16, 2); else if (p.G == 4) MF_AV(16, 4); else MF_AV(16, 8);
+  }
+#undef MF_AV
   return cudaGetLastError();
 }
 

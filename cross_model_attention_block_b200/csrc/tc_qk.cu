@@ -248,28 +248,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&sm.s_empty[sb]);
 
-      // logits in log2 units with band bias and causal mask
+      // Logits in log2 units: x = s * scale2 (+ bias2 in the band), -inf above
+      // the diagonal.  Tiles away from the band and the diagonal ("plain",
+      // most of them) keep raw s and fold the scale into one FMA per element.
       const int kbase = kt * kTile;
-      const bool band_tile = (row0 + kTile - 1) - kbase >= 0 && row0 - (kbase + kTile - 1) < W;
+      const bool band_tile = row0 - (kbase + kTile - 1) < W;
       const bool diag = kt == t;
+      const bool plain = !band_tile && !diag;
+      const float sc = plain ? p.scale2 : 1.f;
+      if (!plain) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const int j = kbase + c;
-        float x = v[c] * p.scale2;
-        if (band_tile && ri - j < W) x += p.bias2;
-        if (diag && j > ri) x = -CUDART_INF_F;
-        v[c] = x;
+        for (int c = 0; c < 128; ++c) {
+          const int j = kbase + c;
+          float x = v[c] * p.scale2;
+          if (ri - j < W) x += p.bias2;
+          if (j > ri) x = -CUDART_INF_F;
+          v[c] = x;
+        }
       }
       if (MODE == kStats) {
-        float mt = -CUDART_INF_F;
+        // tree max and eight independent partial sums (short dependency chains)
+        float mx[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mt = fmaxf(mt, v[c]);
+        for (int k = 0; k < 8; ++k) mx[k] = v[k];
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], v[c + k]);
+        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
         const float m_new = valid ? fmaxf(m_run, mt) : 0.f;
-        float s0 = 0.f, s1 = 0.f;
+        float acc[8];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) s0 += ex2(v[c] - m_new);
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
 #pragma unroll
-        for (int c = 64; c < 128; ++c) s1 += ex2(v[c] - m_new);
+        for (int c = 0; c < 128; c += 8)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[(c >= 64 ? 4 : 0) + (k & 3)] += ex2(fmaf(v[c + k], sc, -m_new));
+        const float s0 = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        const float s1 = (acc[4] + acc[5]) + (acc[6] + acc[7]);
         l_run = l_run * ex2(m_run - m_new) + s0 + s1;
         m_run = m_new;
         if (BB == 128) {
@@ -281,34 +298,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st2(lane_addr + kAcol + 2 * kt, a0, a1);
         }
       } else {
-        // Extraction.  The tile's kept blocks are staged in out[n & 1] as
-        // 128-byte-swizzled [rows][64 keys] sub-tiles and written by TMA
-        // stores: sub-tile b (keys 64b..) for B = 128, (row half a, key half
-        // b) for B = 64.  A row writes only into blocks of its own query
-        // block (which must exist) that are kept.
+        // Extraction.  Each kept block of the tile is staged in out[n & 1] in
+        // the cache's own layout for this head -- one 128-byte line per (key
+        // group, 8-row slice, half), 16-byte chunks permuted by h % 8 -- and
+        // written with one TMA store of those lines.  B = 128: the tile is one
+        // block (256 lines); B = 64: sub-block (row half a, key half b) holds
+        // 64 lines at 8 KB * (2a + b).  A row writes only into kept blocks of
+        // its own query block (which must exist).
+        constexpr int S = BB / 16;
         uint8_t* obuf = sm.out[n & 1];
         if (threadIdx.x == 128) bulk_wait_read<1>();  // stores of tile n-2 done reading
         named_sync_epilogue();
-        const int rr = (BB == 128) ? r : (r & 63);
+        const int rb = r & (BB - 1);  // row within the block
+        const int lrow = ((rb >> 3) << 1) + ((rb & 7) >> 2);  // line of this row, key group 0
+        const int cbase = (rb & 3) << 1;                       // chunk of keys 0-7
         const bool row_ok = qb_r < nqb_s;
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          const int kb = (BB == 128) ? kt : 2 * kt + b;
+        for (int b = 0; b < kTile / BB; ++b) {
+          const int kb = kt * (kTile / BB) + b;
           if (!row_ok || kb > qb_r || p.slot[cb + int64_t(qb_r) * (qb_r + 1) / 2 + kb] < 0)
             continue;
-          uint8_t* sub = obuf + ((BB == 128) ? b * kHalfBytes : ((r >> 6) * 2 + b) * 8192);
+          uint8_t* sub = obuf + ((BB == 128) ? 0 : ((r >> 6) * 2 + b) * 8192);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t w4[4];
+          for (int kg = 0; kg < S; ++kg) {
+            uint8_t* line = sub + (kg * (BB / 4) + lrow) * 128;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float x0 = v[b * 64 + c * 8 + 2 * k], x1 = v[b * 64 + c * 8 + 2 * k + 1];
-              __nv_bfloat162 pr = __floats2bfloat162_rn(valid ? ex2(x0 - lse2) : 0.f,
-                                                        valid ? ex2(x1 - lse2) : 0.f);
-              w4[k] = *reinterpret_cast<uint32_t*>(&pr);
+            for (int c = 0; c < 2; ++c) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int col = b * BB + kg * 16 + c * 8 + 2 * k;
+                __nv_bfloat162 pr =
+                    __floats2bfloat162_rn(valid ? ex2(fmaf(v[col], sc, -lse2)) : 0.f,
+                                          valid ? ex2(fmaf(v[col + 1], sc, -lse2)) : 0.f);
+                w4[k] = *reinterpret_cast<uint32_t*>(&pr);
+              }
+              *reinterpret_cast<uint4*>(line + (((cbase | c) ^ (h & 7)) << 4)) =
+                  make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            *reinterpret_cast<uint4*>(sub + rr * 128 + ((c ^ (rr & 7)) << 4)) =
-                make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
         fence_proxy_async_smem();
@@ -319,14 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int qb = (BB == 128) ? t : 2 * t + a;
             if (qb >= nqb_s) continue;
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-              const int kb = (BB == 128) ? kt : 2 * kt + b;
+            for (int b = 0; b < kTile / BB; ++b) {
+              const int kb = kt * (kTile / BB) + b;
               if (kb > qb) continue;
               const int64_t e = p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kb];
               if (e < 0) continue;
-              const uint8_t* sub = obuf + ((BB == 128) ? b * kHalfBytes : (a * 2 + b) * 8192);
-              tma_store_2d(&tmV, sub, (BB == 128) ? b * 64 : 0,
-                           int32_t((e * p.Hs + h) * BB));
+              const uint8_t* sub = obuf + ((BB == 128) ? 0 : (a * 2 + b) * 8192);
+              tma_store_4d(&tmV, sub, 0, h, 0, int32_t(e));
             }
           }
           bulk_commit();
@@ -448,12 +474,18 @@ static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, c
   if (e != cudaSuccess) return e;
   e = make_tmap_2d_bf16(&tk, K, uint64_t(sz.ntok), cols, 64, qk::kTile, true);
   if (e != cudaSuccess) return e;
-  CUtensorMap tv;  // the cache values as [capacity * Hs * B rows][B keys] (extraction only)
+  // the cache values viewed as (64 elements of a line, head, line (key group,
+  // 8-row slice, half) of an entry, entry): one store writes all lines of one
+  // (entry, head) -- extraction only
+  CUtensorMap tv;
   memset(&tv, 0, sizeof(tv));
   if (mode == qk::kExtract) {
     if (capacity < 1) return cudaSuccess;
-    e = make_tmap_2d_bf16(&tv, values, uint64_t(capacity) * d.Hs * d.B, uint64_t(d.B), 64,
-                          uint32_t(d.B), true);
+    const uint64_t nl = uint64_t(d.B) * uint64_t(d.B) / 64;  // lines per (entry, head)
+    const uint64_t dims[4] = {64, uint64_t(d.Hs), nl, uint64_t(capacity)};
+    const uint64_t strides[3] = {128, uint64_t(d.Hs) * 128, nl * uint64_t(d.Hs) * 128};
+    const uint32_t box[4] = {64, 1, uint32_t(nl), 1};
+    e = make_tmap_bf16(&tv, values, 4, dims, strides, box, 0);
     if (e != cudaSuccess) return e;
   }
   qk::Params p{};

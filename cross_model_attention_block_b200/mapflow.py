@@ -25,7 +25,9 @@ MF_BF16, MF_F32 = 0, 1
 
 EXPORTED = [
     "mf_version", "mf_last_error", "mf_layout_sizes", "mf_block_stats_workspace",
-    "mf_block_stats", "mf_select_extract_workspace", "mf_select_extract", "mf_mapped_av",
+    "mf_block_stats", "mf_select_extract_workspace", "mf_select_extract",
+    "mf_mapped_av_workspace", "mf_mapped_av", "mf_block_stats_noalloc",
+    "mf_block_stats_noalloc_max_workspace",
     "mf_sync_status", "mf_prefix_hash", "mf_index_create", "mf_index_destroy",
     "mf_index_insert", "mf_index_lookup", "mf_index_size",
 ]
@@ -79,7 +81,10 @@ def load_library(path: str = LIB_PATH):
         "mf_block_stats": (C.c_int, [P, P, P, P, P, P, SZ, P]),
         "mf_select_extract_workspace": (SZ, [P]),
         "mf_select_extract": (C.c_int, [P, P, P, P, P, C.c_double, P, P, SZ, P]),
-        "mf_mapped_av": (C.c_int, [P, P, I32, P, P, P, P]),
+        "mf_mapped_av_workspace": (SZ, [P, P, I32, P]),
+        "mf_mapped_av": (C.c_int, [P, P, I32, P, P, P, P, SZ, P]),
+        "mf_block_stats_noalloc_max_workspace": (SZ, []),
+        "mf_block_stats_noalloc": (C.c_int, [P, P, P, P, P, P]),
         "mf_sync_status": (C.c_int, [P]),
         "mf_prefix_hash": (C.c_int, [P, I64, I32, C.c_uint64, P]),
         "mf_index_create": (C.c_int, [P]),
@@ -217,9 +222,11 @@ class Cache:
         return int(self.row_ptr[-1].item())
 
     def values_view(self):
-        """values as [capacity, Hs, B rows, B keys] (see the C header)."""
+        """values in stored order [capacity, B/16 key groups, B/8 row slices, 2 halves,
+        Hs, 8 chunks, 8] (see the C header for the chunk permutation)."""
         B, Hs = self.ctx.B, self.ctx.Hs
-        return self.values[: self.capacity * B * B * Hs].view(self.capacity, Hs, B, B)
+        return self.values[: self.capacity * B * B * Hs].view(
+            self.capacity, B // 16, B // 8, 2, Hs, 8, 8)
 
 
 def select_extract(ctx: Context, Q, K, lse, mass, tau, cache: Cache | None = None):
@@ -239,8 +246,12 @@ def select_extract(ctx: Context, Q, K, lse, mass, tau, cache: Cache | None = Non
     return cache
 
 
-def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None):
-    """Stage 3: O [ntok, Hr, d] = (W-mixed kept map) x V (fused)."""
+def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None,
+              workspace=None):
+    """Stage 3: O [ntok, Hr, d] = (W-mixed kept map) x V (fused).
+
+    `workspace` may be a uint8 device tensor reused across calls (grown when
+    too small); by default one is allocated per call."""
     L = load_library()
     ctx = cache.ctx
     d = ctx.desc()
@@ -251,8 +262,17 @@ def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None
     vd = VDesc(V.data_ptr(), 0 if page_table is None else page_table.data_ptr(),
                page_size, maxp, npages, Hkv, ctx.d)
     cs = cache.struct()
+    nbytes = L.mf_mapped_av_workspace(C.byref(cs), C.byref(d), int(Hr), C.byref(vd))
+    if nbytes == 0:
+        _check(MF_ERR_INVALID_ARG)
+    if workspace is not None and workspace.numel() >= nbytes + 256:
+        ws = workspace
+        wsp = ws.data_ptr() + (-ws.data_ptr()) % 256
+    else:
+        ws, wsp = _workspace(nbytes, W.device)
     _check(L.mf_mapped_av(C.byref(cs), C.byref(d), int(Hr), _ptr(W), C.byref(vd), _ptr(O),
-                          _stream()))
+                          C.c_void_p(wsp), nbytes, _stream()))
+    cache._av_ws = ws  # keep the workspace alive until the stream has used it
     return O
 
 

@@ -84,8 +84,12 @@ typedef struct {
  *          global query block.
  *  values: kept probability blocks P_h[i,j] = exp(s_h[i,j] - lse_h[i]) for
  *          j <= i (0 above the diagonal and beyond the sequence end), of
- *          dtype dt, layout [nnz][Hs][B][B]: entry e, head h, row i of the
- *          query block, key j of the key block (head-major planes).
+ *          dtype dt.  Layout [nnz][B/16][B/8][2][Hs][64]: entry e, key group
+ *          j/16, row slice i/8, half (i%8)/4, head h, then 64 elements of the
+ *          pairs m = (i%4)*16 + j%16 in which the 8-element chunk m/8 is
+ *          stored at chunk (m/8) ^ (h%8) (element m%8 inside it).  One
+ *          (entry, key group, row slice) is Hs * 128 contiguous elements:
+ *          the unit the fused kernel reads.
  *  cu_seqlens, nseq: the context the cache was built from (device). */
 typedef struct {
   int64_t nqb_total;
@@ -107,8 +111,7 @@ typedef struct {
  *  otherwise V is a page pool [npages][page_size][Hkv][d] and
  *  page_table[s * max_pages_per_seq + p] is the pool page holding tokens
  *  p*page_size .. of sequence s; the pool holds npages pages.  page_size
- *  must be a multiple of 16.  Rows of a last page past its sequence's end
- *  must hold finite values (they are multiplied by zero). */
+ *  must be a multiple of 16.  Rows past a sequence's end are never read. */
 typedef struct {
   const void* V;
   const int32_t* page_table;
@@ -192,10 +195,14 @@ mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void*
  *  desc: the sender context (cu_seqlens, Hs, B, dt as in the cache).
  *  W [Hr][Hs] of dtype dt (device); O [ntok][Hr][d] of dtype dt (device, out;
  *  every row of every sequence is written).  No renormalisation of the kept
- *  map.  Hr must be a multiple of Hkv. */
+ *  map.  Hr must be a multiple of Hkv.
+ *  ws: device workspace of at least mf_mapped_av_workspace(...) bytes; it
+ *  holds V regrouped per 16 keys in the tensor cores' operand layout. */
+size_t mf_mapped_av_workspace(const mf_csr_cache* cache, const mf_attn_desc* desc,
+                              int32_t Hr, const mf_v_desc* v);
 mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc,
                        int32_t Hr, const void* W, const mf_v_desc* v, void* O,
-                       mf_stream_t stream);
+                       void* ws, size_t ws_bytes, mf_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the device status word of the
  * current device: MF_OK, MF_ERR_TIMEOUT or MF_ERR_CAPACITY. */

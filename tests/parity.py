@@ -123,7 +123,7 @@ def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
         # extracted probability blocks
         if check_values:
             for e, kb in zip(range(rp[g], rp[g + 1]), kept_g):
-                got = f64(vals[e])                       # [Hs, B rows, B keys]
+                got = stored_to_logical(f64(vals[e]), ctx.Hs, B)  # [Hs, B rows, B keys]
                 ref = np.zeros((P.shape[0], B, B))
                 hi = min(P.shape[2], (kb + 1) * B)
                 ref[:, : i1 - i0, : hi - kb * B] = P[:, :, kb * B:hi]
@@ -140,6 +140,32 @@ def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
         worst = max(worst, err)
         assert err <= tol, f"O seq {s} qb {qb}: rel err {err:.3e} > {tol}"
     return len(picks), n_ex, worst
+
+
+def stored_to_logical(x, Hs, B):
+    """One cache entry, stored [B/16 kg][B/8 slice][2 half][Hs][8 chunk][8] ->
+    logical [Hs][B rows][B keys] (see the C header)."""
+    S16, S8 = B // 16, B // 8
+    x = x.reshape(S16, S8, 2, Hs, 8, 8)
+    out = np.empty((Hs, B, B), dtype=x.dtype)
+    for h in range(Hs):
+        perm = np.arange(8) ^ (h & 7)                 # logical chunk -> stored chunk
+        ch = x[:, :, :, h][:, :, :, perm]             # [kg, slice, half, chunk, 8]
+        ch = ch.reshape(S16, S8, 2, 4, 2, 8)          # chunk = (row % 4, 8-key half)
+        out[h] = ch.transpose(1, 2, 3, 0, 4, 5).reshape(B, B)
+    return out
+
+
+def logical_to_stored(y, Hs, B):
+    """One cache entry, logical [Hs][B][B] -> stored [B/16][B/8][2][Hs][8][8]."""
+    S16, S8 = B // 16, B // 8
+    out = np.empty((S16, S8, 2, Hs, 8, 8), dtype=y.dtype)
+    for h in range(Hs):
+        perm = np.arange(8) ^ (h & 7)
+        blk = y[h].reshape(S8, 2, 4, S16, 2, 8).transpose(3, 0, 1, 2, 4, 5)
+        blk = blk.reshape(S16, S8, 2, 8, 8)           # [kg, slice, half, chunk, 8]
+        out[:, :, :, h][:, :, :, perm] = blk
+    return out
 
 
 def all_picks(ctx):

@@ -94,10 +94,36 @@ def test_argument_errors_return_before_any_launch(lib):
     # mapped AV: Hr must be a multiple of Hkv; page size rule
     v = mfb.VDesc(16, None, 16, 0, 0, 3, 64)
     assert lib.mf_mapped_av(C.byref(cache), C.byref(dsc), 4, P(16), C.byref(v), P(16),
-                            None) == mfb.MF_ERR_INVALID_ARG
+                            P(256), 1 << 20, None) == mfb.MF_ERR_INVALID_ARG
+    assert lib.mf_mapped_av_workspace(C.byref(cache), C.byref(dsc), 4, C.byref(v)) == 0
     v = mfb.VDesc(16, 16, 8, 64, 10, 2, 64)
     assert lib.mf_mapped_av(C.byref(cache), C.byref(dsc), 4, P(16), C.byref(v), P(16),
-                            None) == mfb.MF_ERR_INVALID_ARG
+                            P(256), 1 << 20, None) == mfb.MF_ERR_INVALID_ARG
+    # bf16, d = 128 runs on the tensor-core kernel, which needs a workspace
+    dsc2, host2 = _desc(Hs=40, d=128, B=128, cu=(0, 1000), dt=mfb.MF_BF16)
+    cache2 = mfb.CsrCache(8, 36, 16, 16, 16, 16, 16, 40, 128, mfb.MF_BF16, 1, 0x1000)
+    v2 = mfb.VDesc(16, None, 16, 0, 0, 8, 128)
+    need = lib.mf_mapped_av_workspace(C.byref(cache2), C.byref(dsc2), 32, C.byref(v2))
+    assert need >= 63 * 4096 * 8  # V regrouped per 16 keys: ceil(1000/16) images
+    assert lib.mf_mapped_av(C.byref(cache2), C.byref(dsc2), 32, P(16), C.byref(v2), P(16),
+                            P(256), need - 1, None) == mfb.MF_ERR_WORKSPACE
+
+
+def test_cache_layout_helpers_match_the_header_formula():
+    """tests/parity.py's stored <-> logical transforms follow the C header."""
+    from tests import parity as par
+    for Hs, B in ((8, 64), (40, 128)):
+        y = np.arange(Hs * B * B, dtype=np.float64).reshape(Hs, B, B)
+        st = par.logical_to_stored(y, Hs, B)
+        np.testing.assert_array_equal(par.stored_to_logical(st, Hs, B), y)
+        flat = st.reshape(-1)
+        rng = np.random.default_rng(0)
+        for _ in range(300):
+            h, i, j = int(rng.integers(Hs)), int(rng.integers(B)), int(rng.integers(B))
+            line = (((j // 16) * (B // 8) + i // 8) * 2 + (i % 8) // 4) * Hs + h
+            m = (i % 4) * 16 + j % 16
+            off = line * 64 + ((m // 8) ^ (h % 8)) * 8 + m % 8
+            assert flat[off] == y[h, i, j]
 
 
 # ----------------------------------------------------------- prefix hashing

@@ -201,7 +201,8 @@ def test_mapped_av_on_an_oracle_built_cache(case):
     cache.row_ptr.copy_(torch.tensor(rows, dtype=torch.int64))
     cache.col_idx[: len(cols)].copy_(torch.tensor(cols, dtype=torch.int32))
     vv = cache.values_view()
-    vv[: len(vals)].copy_(torch.from_numpy(np.stack(vals)).to(torch.bfloat16))
+    stored = np.stack([par.logical_to_stored(v, w.Hs, w.B) for v in vals])
+    vv[: len(vals)].copy_(torch.from_numpy(stored).to(torch.bfloat16))
     O = mfb.mapped_av(cache, w.Hr, x.W.cuda(), x.V.cuda(), w.Hkv)
     mfb.sync_status()
     O = O.double().cpu().numpy()

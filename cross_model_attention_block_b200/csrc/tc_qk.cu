@@ -13,9 +13,10 @@
 //  * Extraction: for every kept block of the tile, P = 2^(x - lse2) rounded to
 //    bf16 and written in the cache layout.
 //
-// Roles (256 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
-// tcgen05.mma from one thread, warps 4..7 (one per TMEM lane quarter, one
-// query row per thread) run the epilogue.  S = Q K^T for a 128 x 128 tile
+// Roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// tcgen05.mma from one thread, warps 4..11 run the epilogue as two
+// warpgroups that take turns on the tiles (group n % 2 reads S buffer n % 2),
+// one query row per thread.  S = Q K^T for a 128 x 128 tile
 // lands in one of two TMEM buffers (columns 0..255) so the next tile's MMA
 // overlaps this tile's epilogue; K tiles stream through a 3-stage ring.
 #include <cuda.h>
@@ -36,7 +37,7 @@ namespace qk {
 constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kStages = 3;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // warps 0-3 roles, 4-11 epilogue (two per lane quarter)
 constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB: two [128][64] swizzled halves
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 constexpr uint32_t kTmemCols = 512;
@@ -52,7 +53,8 @@ struct Smem {
   // extraction: two staging tiles for TMA stores, each either two [128][64]
   // (B = 128) or four [64][64] (B = 64) bf16 sub-tiles, 128-byte swizzled
   uint8_t out[2][kTileBytes];
-  float red[4][32];
+  float red[2][4][32];
+  float2 xch[4][64];  // per-row (max, sum) exchange between the two warpgroups
   uint64_t q_full;
   uint64_t k_full[kStages];
   uint64_t k_empty[kStages];
@@ -118,16 +120,40 @@ __device__ __forceinline__ float transpose_reduce32(float* v, int lane) {
 }
 
 __device__ __forceinline__ void named_sync_epilogue() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
-// AND of a predicate over the 128 epilogue threads (named barrier 1).
+// One epilogue warpgroup (named barriers 6, 7).
+__device__ __forceinline__ void group_sync(int wg) {
+  asm volatile("bar.sync %0, 128;" ::"r"(6 + wg) : "memory");
+}
+
+// AND of a predicate over one epilogue warpgroup (named barriers 6, 7).
+__device__ __forceinline__ bool group_all(int wg, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v)), "r"(6 + wg)
+      : "memory");
+  return r != 0;
+}
+
+// The two epilogue warps of one TMEM lane quarter (named barriers 2..5).
+__device__ __forceinline__ void pair_sync(int quarter) {
+  asm volatile("bar.sync %0, 64;" ::"r"(2 + quarter) : "memory");
+}
+
+// AND of a predicate over the 256 epilogue threads (named barrier 1).
 __device__ __forceinline__ bool epilogue_all(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"(uint32_t(v))
@@ -220,13 +246,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
+    // Two warpgroups take turns: group wg handles the tiles n with n % 2 == wg
+    // (S buffer wg), so one group's TMEM reads and exponentials overlap the
+    // other's.  One query row per thread, the 128 columns in two 64-column
+    // chunks.  Key blocks of different tiles are disjoint, so the groups only
+    // merge their row (max, sum) once, at the end.
+    const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // tile row
     const int ri = row0 + r;            // row within the sequence
     const bool valid = ri < L;
     const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
     const int W = p.band_width;
-    float m_run = -CUDART_INF_F, l_run = 0.f;
+    const bool leader = (threadIdx.x & 127) == 0;  // lane 0 of the group's first warp
+    float m_run = -CUDART_INF_F, l_run = 0.f;  // this group's online max and sum
     float lse2 = 0.f;
     if (MODE == kExtract) lse2 = valid ? p.lse[int64_t(h) * p.ntok + seq0 + ri] * kLog2e : 0.f;
     const int qb_r = (BB == 128) ? t : 2 * t + (r >> 6);
@@ -235,121 +268,136 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kt = 0; kt <= t; ++kt) {
       if (!tile_needed<MODE, BB>(p, s, t, kt, nqb_s)) continue;
-      const int sb = n & 1;
+      if ((n & 1) != wg) { ++n; continue; }
+      const int sb = wg;
       bool got = mbar_wait(&sm.s_full[sb], (n >> 1) & 1, p.status);
-      // extraction takes named barriers inside the loop: leave it together
-      if (MODE == kExtract) got = epilogue_all(got);
+      // the loop takes named barriers (extraction staging): leave it together
+      got = group_all(wg, got);
       if (!got) { ok = false; break; }
       tc_fence_after();
-      float v[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + sb * 128 + c * 32, v + c * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&sm.s_empty[sb]);
-
-      // Logits in log2 units: x = s * scale2 (+ bias2 in the band), -inf above
-      // the diagonal.  Tiles away from the band and the diagonal ("plain",
-      // most of them) keep raw s and fold the scale into one FMA per element.
-      const int kbase = kt * kTile;
-      const bool band_tile = row0 - (kbase + kTile - 1) < W;
+      const int kbase0 = kt * kTile;
+      const bool band_tile = row0 - (kbase0 + kTile - 1) < W;
       const bool diag = kt == t;
       const bool plain = !band_tile && !diag;
       const float sc = plain ? p.scale2 : 1.f;
-      if (!plain) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int j = kbase + c;
-          float x = v[c] * p.scale2;
-          if (ri - j < W) x += p.bias2;
-          if (j > ri) x = -CUDART_INF_F;
-          v[c] = x;
-        }
+      uint8_t* obuf = sm.out[wg];
+      if (MODE == kExtract) {
+        if (leader) bulk_wait_read<0>();  // this group's previous stores are done reading
+        group_sync(wg);
       }
-      if (MODE == kStats) {
-        // tree max and eight independent partial sums (short dependency chains)
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = v[k];
-#pragma unroll
-        for (int c = 8; c < 128; c += 8)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], v[c + k]);
-        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
-        const float m_new = valid ? fmaxf(m_run, mt) : 0.f;
-        float acc[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
-#pragma unroll
-        for (int c = 0; c < 128; c += 8)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) acc[(c >= 64 ? 4 : 0) + (k & 3)] += ex2(fmaf(v[c + k], sc, -m_new));
-        const float s0 = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        const float s1 = (acc[4] + acc[5]) + (acc[6] + acc[7]);
-        l_run = l_run * ex2(m_run - m_new) + s0 + s1;
-        m_run = m_new;
-        if (BB == 128) {
-          float a = valid ? m_new + lg2(s0 + s1) : -CUDART_INF_F;
-          tmem_st1(lane_addr + kAcol + kt, a);
-        } else {
-          float a0 = valid ? m_new + lg2(s0) : -CUDART_INF_F;
-          float a1 = valid ? m_new + lg2(s1) : -CUDART_INF_F;
-          tmem_st2(lane_addr + kAcol + 2 * kt, a0, a1);
+      float cm = 0.f, cs = 0.f;  // chunk 0 (max, sum) for a 128-key block
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+        float v[64];
+        tmem_ld32(lane_addr + sb * 128 + ch * 64, v);
+        tmem_ld32(lane_addr + sb * 128 + ch * 64 + 32, v + 32);
+        tmem_wait_ld();
+        if (ch == 1) {
+          tc_fence_before();
+          mbar_arrive(&sm.s_empty[sb]);
         }
-      } else {
-        // Extraction.  Each kept block of the tile is staged in out[n & 1] in
-        // the cache's own layout for this head -- one 128-byte line per (key
-        // group, 8-row slice, half), 16-byte chunks permuted by h % 8 -- and
-        // written with one TMA store of those lines.  B = 128: the tile is one
-        // block (256 lines); B = 64: sub-block (row half a, key half b) holds
-        // 64 lines at 8 KB * (2a + b).  A row writes only into kept blocks of
-        // its own query block (which must exist).
-        constexpr int S = BB / 16;
-        uint8_t* obuf = sm.out[n & 1];
-        if (threadIdx.x == 128) bulk_wait_read<1>();  // stores of tile n-2 done reading
-        named_sync_epilogue();
-        const int rb = r & (BB - 1);  // row within the block
-        const int lrow = ((rb >> 3) << 1) + ((rb & 7) >> 2);  // line of this row, key group 0
-        const int cbase = (rb & 3) << 1;                       // chunk of keys 0-7
-        const bool row_ok = qb_r < nqb_s;
+        // Logits in log2 units: x = s * scale2 (+ bias2 in the band), -inf
+        // above the diagonal.  Tiles away from the band and the diagonal
+        // ("plain", most of them) keep raw s and fold the scale into one FMA.
+        const int kbase = kbase0 + ch * 64;  // key of v[0]
+        if (!plain) {
 #pragma unroll
-        for (int b = 0; b < kTile / BB; ++b) {
-          const int kb = kt * (kTile / BB) + b;
-          if (!row_ok || kb > qb_r || p.slot[cb + int64_t(qb_r) * (qb_r + 1) / 2 + kb] < 0)
-            continue;
-          uint8_t* sub = obuf + ((BB == 128) ? 0 : ((r >> 6) * 2 + b) * 8192);
+          for (int c = 0; c < 64; ++c) {
+            const int j = kbase + c;
+            float x = v[c] * p.scale2;
+            if (ri - j < W) x += p.bias2;
+            if (j > ri) x = -CUDART_INF_F;
+            v[c] = x;
+          }
+        }
+        if (MODE == kStats) {
+          // tree max and eight independent partial sums (short dependency chains)
+          float mx[8];
 #pragma unroll
-          for (int kg = 0; kg < S; ++kg) {
-            uint8_t* line = sub + (kg * (BB / 4) + lrow) * 128;
+          for (int k = 0; k < 8; ++k) mx[k] = v[k];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              uint32_t w4[4];
+          for (int c = 8; c < 64; c += 8)
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int col = b * BB + kg * 16 + c * 8 + 2 * k;
-                __nv_bfloat162 pr =
-                    __floats2bfloat162_rn(valid ? ex2(fmaf(v[col], sc, -lse2)) : 0.f,
-                                          valid ? ex2(fmaf(v[col + 1], sc, -lse2)) : 0.f);
-                w4[k] = *reinterpret_cast<uint32_t*>(&pr);
+            for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], v[c + k]);
+          const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
+          const float m_new = valid ? fmaxf(m_run, mt) : 0.f;
+          // only masked keys seen so far (m = -inf): sum nothing
+          const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
+          float acc[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+#pragma unroll
+          for (int c = 0; c < 64; c += 8)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] += ex2(fmaf(v[c + k], sc, -m_use));
+          const float sh = ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
+                           ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+          l_run = l_run * ex2(m_run - m_use) + sh;
+          m_run = m_new;
+          if (BB == 64) {
+            // each chunk is one key block
+            const float a = valid ? m_new + lg2(sh) : -CUDART_INF_F;
+            tmem_st1(lane_addr + kAcol + 2 * kt + ch, a);
+          } else if (ch == 0) {
+            cm = m_new;
+            cs = sh;
+          } else {
+            // the 128-key block: both chunks relative to the newer max
+            const float tot = cs * ex2(cm - m_use) + sh;
+            const float a = valid ? m_new + lg2(tot) : -CUDART_INF_F;
+            tmem_st1(lane_addr + kAcol + kt, a);
+          }
+        } else {
+          // Extraction into the group's staging tile, in the cache's own layout
+          // for this head: one 128-byte line per (key group, 8-row slice,
+          // half), 16-byte chunks permuted by h % 8.  B = 128: the tile is one
+          // block (256 lines), this chunk fills key groups 4*ch..; B = 64:
+          // sub-block (row half, key half = ch) holds 64 lines at
+          // 8 KB * (2 * rowhalf + ch).  A row writes only into kept blocks of
+          // its own query block (which must exist).
+          const int rb = r & (BB - 1);                          // row within the block
+          const int lrow = ((rb >> 3) << 1) + ((rb & 7) >> 2);  // line of this row, key group 0
+          const int cbase = (rb & 3) << 1;                       // chunk of keys 0-7
+          const int kb = (BB == 128) ? kt : 2 * kt + ch;
+          if (qb_r < nqb_s && kb <= qb_r &&
+              p.slot[cb + int64_t(qb_r) * (qb_r + 1) / 2 + kb] >= 0) {
+            uint8_t* sub = obuf + ((BB == 128) ? 0 : ((r >> 6) * 2 + ch) * 8192);
+#pragma unroll
+            for (int kgl = 0; kgl < 4; ++kgl) {
+              const int kg = (BB == 128) ? ch * 4 + kgl : kgl;
+              uint8_t* line = sub + (kg * (BB / 4) + lrow) * 128;
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const int col = kgl * 16 + c * 8 + 2 * k;
+                  __nv_bfloat162 pr =
+                      __floats2bfloat162_rn(valid ? ex2(fmaf(v[col], sc, -lse2)) : 0.f,
+                                            valid ? ex2(fmaf(v[col + 1], sc, -lse2)) : 0.f);
+                  w4[k] = *reinterpret_cast<uint32_t*>(&pr);
+                }
+                *reinterpret_cast<uint4*>(line + (((cbase | c) ^ (h & 7)) << 4)) =
+                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
               }
-              *reinterpret_cast<uint4*>(line + (((cbase | c) ^ (h & 7)) << 4)) =
-                  make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
           }
         }
+      }
+      if (MODE == kExtract) {
         fence_proxy_async_smem();
-        named_sync_epilogue();
-        if (threadIdx.x == 128) {
+        group_sync(wg);
+        if (leader) {
 #pragma unroll
           for (int a = 0; a < kTile / BB; ++a) {
             const int qb = (BB == 128) ? t : 2 * t + a;
             if (qb >= nqb_s) continue;
 #pragma unroll
             for (int b = 0; b < kTile / BB; ++b) {
-              const int kb = kt * (kTile / BB) + b;
-              if (kb > qb) continue;
-              const int64_t e = p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kb];
+              const int kbb = kt * (kTile / BB) + b;
+              if (kbb > qb) continue;
+              const int64_t e = p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kbb];
               if (e < 0) continue;
               const uint8_t* sub = obuf + ((BB == 128) ? 0 : (a * 2 + b) * 8192);
               tma_store_4d(&tmV, sub, 0, h, 0, int32_t(e));
@@ -360,33 +408,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++n;
     }
-    if (MODE == kExtract && threadIdx.x == 128) bulk_wait_all<0>();
+    if (MODE == kExtract && leader) bulk_wait_all<0>();
     ok = epilogue_all(ok);  // uniform, so every thread takes the named barriers below
     if (MODE == kStats && ok) {
-      lse2 = valid ? m_run + lg2(l_run) : 0.f;
-      if (valid) p.lse[int64_t(h) * p.ntok + seq0 + ri] = lse2 * kLn2;
+      // row log-sum-exp from the two groups' (max, sum)
+      {
+        float2* xs = sm.xch[quarter];
+        xs[wg * 32 + lane] = make_float2(m_run, l_run);
+        pair_sync(quarter);
+        const float2 o = xs[(wg ^ 1) * 32 + lane];
+        const float M = fmaxf(m_run, o.x);
+        const float Mu = M == -CUDART_INF_F ? 0.f : M;
+        const float l = l_run * ex2(m_run - Mu) + o.y * ex2(o.x - Mu);
+        lse2 = valid ? M + lg2(l) : 0.f;
+      }
+      if (valid && wg == 0) p.lse[int64_t(h) * p.ntok + seq0 + ri] = lse2 * kLn2;
       tmem_wait_st();
+      tc_fence_before();
+      named_sync_epilogue();  // both groups' log partials are in TMEM
+      tc_fence_after();
+      // block masses: chunks of 32 key blocks, even chunks to group 0, odd to group 1
       const int nkb = (t + 1) * (kTile / BB);
-      for (int c0 = 0; c0 < nkb; c0 += 32) {
+      for (int c2 = 0; c2 < nkb; c2 += 64) {
+        const int c0 = c2 + wg * 32;
         float a[32];
-        tmem_ld32(lane_addr + kAcol + c0, a);
+        tmem_ld32(lane_addr + kAcol + min(c0, 256 - 32), a);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 32; ++k)
           a[k] = (valid && c0 + k < nkb) ? ex2(a[k] - lse2) : 0.f;
         const float tot = transpose_reduce32(a, lane);
         named_sync_epilogue();
-        sm.red[quarter][lane] = tot;
+        sm.red[wg][quarter][lane] = tot;
         named_sync_epilogue();
-        if (quarter == 0) {
+        if (quarter == 0 && c0 < nkb) {
           const int kb = c0 + lane;
           if (BB == 128) {
-            float m = (sm.red[0][lane] + sm.red[1][lane]) + (sm.red[2][lane] + sm.red[3][lane]);
+            const float m = (sm.red[wg][0][lane] + sm.red[wg][1][lane]) +
+                            (sm.red[wg][2][lane] + sm.red[wg][3][lane]);
             if (kb <= t) p.part[int64_t(h) * p.nblocks + cb + int64_t(t) * (t + 1) / 2 + kb] = m;
           } else {
             const int qa = 2 * t, qbb = 2 * t + 1;
-            float m0 = sm.red[0][lane] + sm.red[1][lane];
-            float m1 = sm.red[2][lane] + sm.red[3][lane];
+            const float m0 = sm.red[wg][0][lane] + sm.red[wg][1][lane];
+            const float m1 = sm.red[wg][2][lane] + sm.red[wg][3][lane];
             if (kb <= qa) p.part[int64_t(h) * p.nblocks + cb + int64_t(qa) * (qa + 1) / 2 + kb] = m0;
             if (qbb < nqb_s && kb <= qbb)
               p.part[int64_t(h) * p.nblocks + cb + int64_t(qbb) * (qbb + 1) / 2 + kb] = m1;

@@ -21,10 +21,11 @@
 //      M^T_g[16 keys x 8 rows * G heads], the MN-major operand of step 3;
 //   3. O MMAs    O^T_g[128 d x 8G] += V_g^T[128 x 16] . M^T_g[16 x 8G] for every
 //      GQA group g (O^T of all groups resident in TMEM for the whole CTA).
-// The four converting warps also drive the tensor core: one of their lanes
-// issues mix(n+1) before stage n is converted and O(n) right after a named
-// barrier closes the conversion, so no stage waits on a hand-off to another
-// warp (an mbarrier round trip costs more than a stage's work).
+// A dedicated MMA warp issues every MMA with descriptors built once (only the
+// address field moves).  Converters hand each stage over through a named
+// barrier (hardware, no mbarrier round trip between warps), and mix(n + 2) is
+// issued as soon as stage n's accumulator has been read, keeping the tensor
+// core ahead of the conversion.
 //
 // Why not mma.sync for the mix: on this part a legacy mma.sync takes a few
 // thousand cycles from issue to result unless hundreds are in flight; with
@@ -76,18 +77,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// AND of a predicate over the 128 worker threads (named barrier 1).
-__device__ __forceinline__ bool epilogue_all(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(uint32_t(v))
-      : "memory");
-  return r != 0;
+// Named barriers 1 and 2 (by stage parity) hand stage n from the converters
+// to the MMA warp: both sides bar.sync once per stage, so neither can run a
+// phase ahead, also when a timed-out wait makes the rest of the walk a no-op.
+constexpr int kBarMt = 1;
+
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Stage walk: (entry e, key group kg) pairs of one query block, skipping key
@@ -140,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   uint64_t* mix_full = vm_empty + VS;                                   // [kMixBufs]
   uint64_t* final_bar = mix_full + kMixBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slices = p.B / kRows;
@@ -162,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     }
     for (int i = 0; i < kMixBufs; ++i) mbar_init(&mix_full[i], 1);
     mbar_init(final_bar, 1);
+    *abort = 0;
     fence_barrier_init();
   }
   // W^T as the K-major operand [Hr rows][Hs_pad], core matrices of 8 rows x 16
@@ -189,6 +187,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(base);
   const int S16 = p.B / 16, S8 = p.B / 8;
+  // a wait that gave up makes every later wait of the CTA give up at once, so
+  // the named-barrier hand-offs below still run to the end without blocking
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (*abort) return false;
+    if (mbar_wait(bar, parity, p.status)) return true;
+    *abort = 1;
+    return false;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------- map producer
@@ -197,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
       int n = 0;
       while (wk.next()) {
         const int st = n % MS;
-        if (!mbar_wait(&map_empty[st], ((n / MS) & 1) ^ 1, p.status)) break;
+        if (!wait(&map_empty[st], ((n / MS) & 1) ^ 1)) break;
         mbar_expect_tx(&map_full[st], p.map_bytes);
         const int64_t line0 = ((wk.e * S16 + wk.kg) * S8 + slice) * 2 * p.Hs;
         bulk_load(base + p.off_map + st * p.map_slot, p.values + line0 * 64, p.map_bytes,
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
       int n = 0;
       while (wk.next()) {
         const int st = n % VS;
-        if (!mbar_wait(&vm_empty[st], ((n / VS) & 1) ^ 1, p.status)) break;
+        if (!wait(&vm_empty[st], ((n / VS) & 1) ^ 1)) break;
         mbar_expect_tx(&v_full[st], p.v_bytes);
         const int64_t grp = g0 + (wk.kb * p.B + wk.kg * kKeys) / kKeys;
         bulk_load(base + p.off_v + st * p.v_bytes, p.vimg + grp * p.v_bytes, p.v_bytes,
@@ -221,93 +227,96 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
         ++n;
       }
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ workers
-    // One lane issues every MMA; all 128 threads (one per mix-accumulator
-    // lane = (row, key) pair) convert.  mix(n+1) is issued before stage n is
-    // converted, so its tensor-core time overlaps the conversion.
-    const int q = warp & 3;  // TMEM lane quarter: pairs 32q .. 32q+31
-    const int m = q * 32 + lane;
-    const int r8 = m >> 4, k16 = m & 15;
-    const bool leader = threadIdx.x == 128;
-    const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA warp
+    // Descriptors are built once; per MMA only the start-address field moves
+    // (added in 16-byte units, never carrying out of its 14 bits).
     const uint32_t idesc_mix = idesc_bf16(128, HR, 1, 0);  // A MN-major, B K-major
     const uint32_t idesc_o = idesc_bf16(128, NO, 1, 1);    // A, B MN-major
     const int ksteps = p.Hs_pad / 16;
-    // mix(n): Mix[pairs x Hr] = Map[pairs x Hs] . W^T into accumulator n % kMixBufs
-    auto issue_mix = [&](int n) -> bool {
+    const uint64_t mix_a0 = smem_desc(sbase + p.off_map, p.Hs * 128, 1024, kSwizzle128);
+    const uint64_t mix_b0 = smem_desc(sbase + p.off_w, 128, p.Hs_pad * 16, kSwizzleNone);
+    const uint64_t o_a0 = smem_desc(sbase + p.off_v, 2048, 1024, kSwizzle128);
+    const uint64_t o_b0 = smem_desc(sbase + p.off_mt, 128, 256, kSwizzleNone);
+    auto issue_mix = [&](int n) {
       const int ms = n % MS;
-      if (!mbar_wait(&map_full[ms], (n / MS) & 1, p.status)) return false;
+      if (!wait(&map_full[ms], (n / MS) & 1)) return;
       tc_fence_after();
-      const uint32_t ma = sbase + p.off_map + ms * p.map_slot;
-      for (int kk = 0; kk < ksteps; ++kk) {
-        // A = map slab: MN-major, 128-byte swizzle, pair halves Hs * 128 B apart,
-        // 8-head groups 1 KB apart; B = W^T: K-major, no swizzle
-        const uint64_t adesc = smem_desc(ma + kk * 2048, p.Hs * 128, 1024, kSwizzle128);
-        const uint64_t bdesc =
-            smem_desc(sbase + p.off_w + kk * 256, 128, p.Hs_pad * 16, kSwizzleNone);
-        mma_bf16_ss(tmem + kMixCol + (n % kMixBufs) * HR, adesc, bdesc, idesc_mix, kk > 0);
-      }
+      const uint64_t a = mix_a0 + ((ms * p.map_slot) >> 4);
+      const uint32_t d = tmem + kMixCol + (n % kMixBufs) * HR;
+      for (int kk = 0; kk < ksteps; ++kk)
+        mma_bf16_ss(d, a + kk * (2048 >> 4), mix_b0 + kk * (256 >> 4), idesc_mix, kk > 0);
       mma_commit(&map_empty[ms]);
       mma_commit(&mix_full[n % kMixBufs]);
-      return true;
     };
     Walk wk = make_walk(p, gqb, L);
     Walk ahead = wk;
-    bool more = ahead.next();  // `ahead` runs one stage in front of `wk`
-    bool lead_ok = true;
-    if (leader && more) lead_ok = issue_mix(0);
+    int navail = 0;  // stages the look-ahead walk has produced
+    if (lane == 0) {
+      for (int k = 0; k < kMixBufs && ahead.next(); ++k) issue_mix(navail++);
+    }
+    navail = __shfl_sync(0xffffffffu, navail, 0);
     int n = 0;
     while (wk.next()) {
-      more = ahead.next();
-      if (leader && more && lead_ok) lead_ok = issue_mix(n + 1);
-      const int db = n % kMixBufs, vs = n % VS;
-      bool ok = mbar_wait(&mix_full[db], (n / kMixBufs) & 1, p.status);
-      tc_fence_after();
-      float v[HR];
-      if constexpr (HR == 32) {
-        tmem_ld32(lane_addr + kMixCol + db * HR, v);
-      } else {
-        tmem_ld16(lane_addr + kMixCol + db * HR, v);
-      }
-      tmem_wait_ld();
-      ok = ok && mbar_wait(&vm_empty[vs], ((n / VS) & 1) ^ 1, p.status);  // M^T slot free
-      const int kvalid = min(kKeys, L - (wk.kb * p.B + wk.kg * kKeys));  // keys < L
-      const float z = (k16 < kvalid && i0 + r8 < L) ? 1.f : 0.f;
-      uint8_t* mt = base + p.off_mt + vs * p.mt_bytes + (k16 >> 3) * 128 + (k16 & 7) * 16;
+      const int vs = n % VS;
+      named_sync(kBarMt + (n & 1), 160);  // stage n's M^T is written, its mix buffer read
+      if (lane == 0) {
+        if (wait(&v_full[vs], (n / VS) & 1)) {
+          tc_fence_after();
+          const uint64_t a = o_a0 + ((vs * p.v_bytes) >> 4);
+          const uint64_t b = o_b0 + ((vs * p.mt_bytes) >> 4);
 #pragma unroll
-      for (int r = 0; r < HR; r += 2) {
-        const int g = r / G, rl = r % G;
-        const int nn = r8 * G + rl;  // MMA N index of (row r8, head r)
-        *reinterpret_cast<uint32_t*>(mt + g * p.mt_group_stride + (nn >> 3) * 256 +
-                                     ((nn & 7) << 1)) = pack_bf16(v[r] * z, v[r + 1] * z);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      // all four warps' M^T (and their reads of accumulator db) are done
-      if (!epilogue_all(ok)) break;
-      if (leader) {
-        // O(n): O^T_g += V_g^T . M^T_g for every GQA group
-        if (!mbar_wait(&v_full[vs], (n / VS) & 1, p.status)) lead_ok = false;
-        tc_fence_after();
-        const uint32_t va = sbase + p.off_v + vs * p.v_bytes;
-        const uint32_t mb = sbase + p.off_mt + vs * p.mt_bytes;
-#pragma unroll
-        for (int g = 0; g < HKV; ++g) {
-          // A = V_g^T: MN-major, 128-byte swizzle, d halves 2 KB apart, 8-key groups 1 KB apart
-          const uint64_t adesc = smem_desc(va + g * 4096, 2048, 1024, kSwizzle128);
-          // B = M^T_g: MN-major, no swizzle, n-chunks 256 B apart, 8-key groups 128 B apart
-          const uint64_t bdesc = smem_desc(mb + g * p.mt_group_stride, 128, 256, kSwizzleNone);
-          if (lead_ok) mma_bf16_ss(tmem + g * NO, adesc, bdesc, idesc_o, n > 0);
+          for (int g = 0; g < HKV; ++g)
+            mma_bf16_ss(tmem + g * NO, a + g * (4096 >> 4), b + g * (p.mt_group_stride >> 4),
+                        idesc_o, n > 0);
         }
         mma_commit(&vm_empty[vs]);
+        if (ahead.next()) issue_mix(navail++);  // into the buffer stage n just freed
       }
       ++n;
     }
-    if (leader) mma_commit(final_bar);
+    if (lane == 0) mma_commit(final_bar);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ converters
+    // One thread per mix-accumulator lane = (row, key) pair.
+    const int q = warp & 3;  // TMEM lane quarter: pairs 32q .. 32q+31
+    const int m = q * 32 + lane;
+    const int r8 = m >> 4, k16 = m & 15;
+    const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
+    Walk wk = make_walk(p, gqb, L);
+    int n = 0;
+    while (wk.next()) {
+      const int db = n % kMixBufs, vs = n % VS;
+      if (wait(&mix_full[db], (n / kMixBufs) & 1)) {
+        tc_fence_after();
+        float v[HR];
+        if constexpr (HR == 32) {
+          tmem_ld32(lane_addr + kMixCol + db * HR, v);
+        } else {
+          tmem_ld16(lane_addr + kMixCol + db * HR, v);
+        }
+        tmem_wait_ld();
+        if (wait(&vm_empty[vs], ((n / VS) & 1) ^ 1)) {  // M^T slot free
+          const int kvalid = min(kKeys, L - (wk.kb * p.B + wk.kg * kKeys));  // keys < L
+          const float z = (k16 < kvalid && i0 + r8 < L) ? 1.f : 0.f;
+          uint8_t* mt = base + p.off_mt + vs * p.mt_bytes + (k16 >> 3) * 128 + (k16 & 7) * 16;
+#pragma unroll
+          for (int r = 0; r < HR; r += 2) {
+            const int g = r / G, rl = r % G;
+            const int nn = r8 * G + rl;  // MMA N index of (row r8, head r)
+            *reinterpret_cast<uint32_t*>(mt + g * p.mt_group_stride + (nn >> 3) * 256 +
+                                         ((nn & 7) << 1)) = pack_bf16(v[r] * z, v[r + 1] * z);
+          }
+          fence_proxy_async_smem();
+        }
+      }
+      tc_fence_before();
+      named_sync(kBarMt + (n & 1), 160);  // hand stage n to the MMA warp
+      ++n;
+    }
     // ------------------------------------------------------------ epilogue
     const int c = q * 32 + lane;  // d index = TMEM lane
-    const bool ok = mbar_wait(final_bar, 0, p.status);
+    const bool ok = wait(final_bar, 0);
     tc_fence_after();
 #pragma unroll 1
     for (int g = 0; g < HKV; ++g) {
@@ -462,7 +471,7 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.off_mt = p.off_map + ms * p.map_slot;
   p.off_w = p.off_mt + vs * p.mt_bytes;
   p.off_bar = (p.off_w + p.w_bytes + 7u) & ~7u;
-  const size_t smem = size_t(p.off_bar) + (2 * ms + 2 * vs + av::kMixBufs + 1) * 8 + 16 + 1024;
+  const size_t smem = size_t(p.off_bar) + (2 * ms + 2 * vs + av::kMixBufs + 1) * 8 + 32 + 1024;
   const unsigned grid = unsigned(sz.nqb) * unsigned(d.B / av::kRows);
   cudaError_t e = cudaSuccess;
 #define MF_AV(HR, G)                                                                        \

@@ -302,6 +302,8 @@ mf_status mf_sync_status(mf_stream_t stream) {
   }
   if (v & kStatusTimeout) return fail(MF_ERR_TIMEOUT, "a device-side bounded wait gave up");
   if (v & kStatusCapacity) return fail(MF_ERR_CAPACITY, "kept blocks exceed nnz_capacity");
+  if (v & kStatusBadCache)
+    return fail(MF_ERR_INVALID_ARG, "a cache row holds more entries than its query block has key blocks");
   return MF_OK;
 }
 

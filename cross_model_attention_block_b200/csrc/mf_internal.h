@@ -11,7 +11,7 @@
 namespace mf {
 
 // Bits of the per-device status word.
-enum : unsigned { kStatusTimeout = 1u, kStatusCapacity = 2u };
+enum : unsigned { kStatusTimeout = 1u, kStatusCapacity = 2u, kStatusBadCache = 4u };
 
 // Device address of the status word of the current device.
 unsigned* status_word();

@@ -48,7 +48,9 @@ constexpr int kD = 128;
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxMapStages = 8;
-constexpr int kMixBufs = 2;  // mix accumulators in TMEM (mix(n+1) runs while n converts)
+// Mix accumulators in TMEM: mix(n + kMixBufs) is issued as soon as stage n has
+// been converted, so kMixBufs stages of MMA latency overlap the conversion.
+constexpr int kMixBufs = 4;
 
 struct Params {
   const int64_t* row_ptr;
@@ -67,7 +69,7 @@ struct Params {
   uint32_t map_bytes;       // Hs * 256 (one stage)
   uint32_t map_slot;        // map_bytes + 1 KB zero guard, 1 KB aligned
   uint32_t v_bytes, mt_group_stride, mt_bytes, w_bytes;
-  uint32_t off_v, off_map, off_mt, off_w, off_bar;
+  uint32_t off_v, off_map, off_mt, off_w, off_kb, off_bar;
   int map_stages, vm_stages;
   unsigned* status;
 };
@@ -86,38 +88,34 @@ __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Stage walk: (entry e, key group kg) pairs of one query block, skipping key
-// groups that start past the sequence end.
-struct Walk {
-  int64_t e, e1;
-  int kg, nkg, kb;
-  int B, L;
-  const int32_t* col_idx;
-  __device__ bool next() {
-    while (true) {
-      if (kg + 1 < nkg) { ++kg; return true; }
-      ++e;
-      if (e >= e1) return false;
-      kb = col_idx[e];
-      const int rem = L - kb * B;
-      nkg = (min(rem, B) + kKeys - 1) / kKeys;
-      kg = -1;
-      if (nkg <= 0) nkg = 0;
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Ring position: slot and the parity of its current use, advanced without
+// division (stage counters never feed a divide in the issue path).
+struct Ring {
+  int slot = 0;
+  uint32_t phase = 0;
+  int size;
+  __device__ explicit Ring(int n) : size(n) {}
+  __device__ void next() {
+    if (++slot == size) {
+      slot = 0;
+      phase ^= 1u;
     }
   }
 };
 
-__device__ __forceinline__ Walk make_walk(const Params& p, int64_t gqb, int L) {
-  Walk w;
-  w.e = p.row_ptr[gqb] - 1;
-  w.e1 = min(p.row_ptr[gqb + 1], p.capacity);
-  w.kg = 0;
-  w.nkg = 0;
-  w.kb = 0;
-  w.B = p.B;
-  w.L = L;
-  w.col_idx = p.col_idx;
-  return w;
+// A stage is (kept entry e, 16-key group kg) of the CTA's query block; key
+// groups that start past the sequence end are skipped.
+__device__ __forceinline__ int key_groups_of(int kb, int B, int L) {
+  const int rem = L - kb * B;
+  return rem <= 0 ? 0 : min(B, rem + kKeys - 1) / kKeys;
 }
 
 template <int HR, int G>
@@ -125,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   constexpr int HKV = HR / G;
   constexpr int NO = kRows * G;          // O MMA N per group
   constexpr uint32_t kMixCol = 8u * HR;  // first TMEM column of the mix accumulators
+  static_assert(kMixCol + kMixBufs * HR <= kTmemCols, "O^T and mix accumulators exceed TMEM");
+  static_assert((kMixBufs & (kMixBufs - 1)) == 0, "kMixBufs must be a power of two");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   uint64_t* final_bar = mix_full + kMixBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_kb = reinterpret_cast<int32_t*>(base + p.off_kb);  // kept key blocks of the row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slices = p.B / kRows;
@@ -147,7 +148,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   const int L = p.cu_seqlens[s + 1] - seq0;
   const int i0 = qb * p.B + slice * kRows;  // first row (in the sequence)
   if (i0 >= L) return;                      // the whole slice is past the sequence end
+  const int64_t e0 = p.row_ptr[gqb];
+  int nE = int(max(int64_t(0), min(p.row_ptr[gqb + 1], p.capacity) - e0));
+  if (nE > qb + 1) {  // a causal row holds at most qb + 1 key blocks
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusBadCache);
+    nE = qb + 1;
+  }
 
+  for (int e = threadIdx.x; e < nE; e += kThreads) s_kb[e] = p.col_idx[e0 + e];
   if (threadIdx.x == 0) {
     for (int i = 0; i < MS; ++i) {
       mbar_init(&map_full[i], 1);
@@ -186,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(base);
-  const int S16 = p.B / 16, S8 = p.B / 8;
+  const int S8 = p.B / 8;
   // a wait that gave up makes every later wait of the CTA give up at once, so
   // the named-barrier hand-offs below still run to the end without blocking
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -199,38 +207,55 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   if (warp == 0) {
     // ------------------------------------------------------- map producer
     if (lane == 0) {
-      Walk wk = make_walk(p, gqb, L);
-      int n = 0;
-      while (wk.next()) {
-        const int st = n % MS;
-        if (!wait(&map_empty[st], ((n / MS) & 1) ^ 1)) break;
-        mbar_expect_tx(&map_full[st], p.map_bytes);
-        const int64_t line0 = ((wk.e * S16 + wk.kg) * S8 + slice) * 2 * p.Hs;
-        bulk_load(base + p.off_map + st * p.map_slot, p.values + line0 * 64, p.map_bytes,
-                  &map_full[st]);
-        ++n;
+      Ring ring(MS);
+      bool live = true;
+      for (int e = 0; e < nE && live; ++e) {
+        const int nk = key_groups_of(s_kb[e], p.B, L);
+        const int64_t line_e = (e0 + e) * (p.B / 16);
+        for (int kg = 0; kg < nk; ++kg) {
+          if (!wait(&map_empty[ring.slot], ring.phase ^ 1u)) {
+            live = false;
+            break;
+          }
+          mbar_expect_tx(&map_full[ring.slot], p.map_bytes);
+          const int64_t line0 = ((line_e + kg) * S8 + slice) * 2 * p.Hs;
+          bulk_load(base + p.off_map + ring.slot * p.map_slot, p.values + line0 * 64,
+                    p.map_bytes, &map_full[ring.slot]);
+          ring.next();
+        }
       }
     }
   } else if (warp == 2) {
     // --------------------------------------------------------- V producer
     if (lane == 0) {
-      Walk wk = make_walk(p, gqb, L);
+      Ring ring(VS);
       const int64_t g0 = p.cu_g[s];
-      int n = 0;
-      while (wk.next()) {
-        const int st = n % VS;
-        if (!wait(&vm_empty[st], ((n / VS) & 1) ^ 1)) break;
-        mbar_expect_tx(&v_full[st], p.v_bytes);
-        const int64_t grp = g0 + (wk.kb * p.B + wk.kg * kKeys) / kKeys;
-        bulk_load(base + p.off_v + st * p.v_bytes, p.vimg + grp * p.v_bytes, p.v_bytes,
-                  &v_full[st]);
-        ++n;
+      bool live = true;
+      for (int e = 0; e < nE && live; ++e) {
+        const int kb = s_kb[e];
+        const int nk = key_groups_of(kb, p.B, L);
+        for (int kg = 0; kg < nk; ++kg) {
+          if (!wait(&vm_empty[ring.slot], ring.phase ^ 1u)) {
+            live = false;
+            break;
+          }
+          mbar_expect_tx(&v_full[ring.slot], p.v_bytes);
+          const int64_t grp = g0 + int64_t(kb) * (p.B / kKeys) + kg;
+          bulk_load(base + p.off_v + ring.slot * p.v_bytes, p.vimg + grp * p.v_bytes, p.v_bytes,
+                    &v_full[ring.slot]);
+          ring.next();
+        }
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA warp
-    // Descriptors are built once; per MMA only the start-address field moves
-    // (added in 16-byte units, never carrying out of its 14 bits).
+    // The whole warp walks the stages (it takes part in the named barriers);
+    // one elected lane issues.  Descriptors are built once, per MMA only the
+    // start-address field moves (added in 16-byte units, never carrying out
+    // of its 14 bits), and ring positions advance without division.
+    int nst = 0;
+    for (int e = lane; e < nE; e += 32) nst += key_groups_of(s_kb[e], p.B, L);
+    nst = __reduce_add_sync(0xffffffffu, nst);
     const uint32_t idesc_mix = idesc_bf16(128, HR, 1, 0);  // A MN-major, B K-major
     const uint32_t idesc_o = idesc_bf16(128, NO, 1, 1);    // A, B MN-major
     const int ksteps = p.Hs_pad / 16;
@@ -238,44 +263,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     const uint64_t mix_b0 = smem_desc(sbase + p.off_w, 128, p.Hs_pad * 16, kSwizzleNone);
     const uint64_t o_a0 = smem_desc(sbase + p.off_v, 2048, 1024, kSwizzle128);
     const uint64_t o_b0 = smem_desc(sbase + p.off_mt, 128, 256, kSwizzleNone);
-    auto issue_mix = [&](int n) {
-      const int ms = n % MS;
-      if (!wait(&map_full[ms], (n / MS) & 1)) return;
+    const uint32_t map_step = p.map_slot >> 4, v_step = p.v_bytes >> 4,
+                   mt_step = p.mt_bytes >> 4, mtg_step = p.mt_group_stride >> 4;
+    Ring mring(MS), vring(VS);
+    auto issue_mix = [&](int m) {
+      const bool ok = __all_sync(0xffffffffu, wait(&map_full[mring.slot], mring.phase));
       tc_fence_after();
-      const uint64_t a = mix_a0 + ((ms * p.map_slot) >> 4);
-      const uint32_t d = tmem + kMixCol + (n % kMixBufs) * HR;
-      for (int kk = 0; kk < ksteps; ++kk)
-        mma_bf16_ss(d, a + kk * (2048 >> 4), mix_b0 + kk * (256 >> 4), idesc_mix, kk > 0);
-      mma_commit(&map_empty[ms]);
-      mma_commit(&mix_full[n % kMixBufs]);
+      if (ok && elect_one()) {
+        const uint64_t a = mix_a0 + uint64_t(mring.slot) * map_step;
+        const uint32_t d = tmem + kMixCol + uint32_t(m & (kMixBufs - 1)) * HR;
+        for (int kk = 0; kk < ksteps; ++kk)
+          mma_bf16_ss(d, a + kk * (2048 >> 4), mix_b0 + kk * (256 >> 4), idesc_mix, kk > 0);
+        mma_commit(&map_empty[mring.slot]);
+        mma_commit(&mix_full[m & (kMixBufs - 1)]);
+      }
+      __syncwarp();
+      mring.next();
     };
-    Walk wk = make_walk(p, gqb, L);
-    Walk ahead = wk;
-    int navail = 0;  // stages the look-ahead walk has produced
-    if (lane == 0) {
-      for (int k = 0; k < kMixBufs && ahead.next(); ++k) issue_mix(navail++);
-    }
-    navail = __shfl_sync(0xffffffffu, navail, 0);
-    int n = 0;
-    while (wk.next()) {
-      const int vs = n % VS;
+    for (int m = 0; m < kMixBufs && m < nst; ++m) issue_mix(m);
+    for (int n = 0; n < nst; ++n) {
       named_sync(kBarMt + (n & 1), 160);  // stage n's M^T is written, its mix buffer read
-      if (lane == 0) {
-        if (wait(&v_full[vs], (n / VS) & 1)) {
-          tc_fence_after();
-          const uint64_t a = o_a0 + ((vs * p.v_bytes) >> 4);
-          const uint64_t b = o_b0 + ((vs * p.mt_bytes) >> 4);
+      const bool ok = __all_sync(0xffffffffu, wait(&v_full[vring.slot], vring.phase));
+      tc_fence_after();
+      if (elect_one()) {
+        if (ok) {
+          const uint64_t a = o_a0 + uint64_t(vring.slot) * v_step;
+          const uint64_t b = o_b0 + uint64_t(vring.slot) * mt_step;
 #pragma unroll
           for (int g = 0; g < HKV; ++g)
-            mma_bf16_ss(tmem + g * NO, a + g * (4096 >> 4), b + g * (p.mt_group_stride >> 4),
-                        idesc_o, n > 0);
+            mma_bf16_ss(tmem + g * NO, a + g * (4096 >> 4), b + uint64_t(g) * mtg_step, idesc_o,
+                        n > 0);
         }
-        mma_commit(&vm_empty[vs]);
-        if (ahead.next()) issue_mix(navail++);  // into the buffer stage n just freed
+        mma_commit(&vm_empty[vring.slot]);
       }
-      ++n;
+      __syncwarp();
+      vring.next();
+      if (n + kMixBufs < nst) issue_mix(n + kMixBufs);  // into the buffer stage n freed
     }
-    if (lane == 0) mma_commit(final_bar);
+    if (elect_one()) mma_commit(final_bar);
+    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ converters
     // One thread per mix-accumulator lane = (row, key) pair.
@@ -283,36 +309,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     const int m = q * 32 + lane;
     const int r8 = m >> 4, k16 = m & 15;
     const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
-    Walk wk = make_walk(p, gqb, L);
+    const bool row_ok = i0 + r8 < L;
+    uint8_t* mt0 = base + p.off_mt + (k16 >> 3) * 128 + (k16 & 7) * 16;
+    Ring vring(VS);
     int n = 0;
-    while (wk.next()) {
-      const int db = n % kMixBufs, vs = n % VS;
-      if (wait(&mix_full[db], (n / kMixBufs) & 1)) {
-        tc_fence_after();
-        float v[HR];
-        if constexpr (HR == 32) {
-          tmem_ld32(lane_addr + kMixCol + db * HR, v);
-        } else {
-          tmem_ld16(lane_addr + kMixCol + db * HR, v);
-        }
-        tmem_wait_ld();
-        if (wait(&vm_empty[vs], ((n / VS) & 1) ^ 1)) {  // M^T slot free
-          const int kvalid = min(kKeys, L - (wk.kb * p.B + wk.kg * kKeys));  // keys < L
-          const float z = (k16 < kvalid && i0 + r8 < L) ? 1.f : 0.f;
-          uint8_t* mt = base + p.off_mt + vs * p.mt_bytes + (k16 >> 3) * 128 + (k16 & 7) * 16;
-#pragma unroll
-          for (int r = 0; r < HR; r += 2) {
-            const int g = r / G, rl = r % G;
-            const int nn = r8 * G + rl;  // MMA N index of (row r8, head r)
-            *reinterpret_cast<uint32_t*>(mt + g * p.mt_group_stride + (nn >> 3) * 256 +
-                                         ((nn & 7) << 1)) = pack_bf16(v[r] * z, v[r + 1] * z);
+    for (int e = 0; e < nE; ++e) {
+      const int kb = s_kb[e];
+      const int nk = key_groups_of(kb, p.B, L);
+      for (int kg = 0; kg < nk; ++kg, ++n) {
+        const int db = n & (kMixBufs - 1);
+        if (wait(&mix_full[db], uint32_t(n / kMixBufs) & 1u)) {
+          tc_fence_after();
+          float v[HR];
+          if constexpr (HR == 32) {
+            tmem_ld32(lane_addr + kMixCol + db * HR, v);
+          } else {
+            tmem_ld16(lane_addr + kMixCol + db * HR, v);
           }
-          fence_proxy_async_smem();
+          tmem_wait_ld();
+          if (wait(&vm_empty[vring.slot], vring.phase ^ 1u)) {  // M^T slot free
+            const int key = kb * p.B + kg * kKeys + k16;
+            const float z = (key < L && row_ok) ? 1.f : 0.f;
+            uint8_t* mt = mt0 + vring.slot * p.mt_bytes;
+#pragma unroll
+            for (int r = 0; r < HR; r += 2) {
+              const int g = r / G, rl = r % G;
+              const int nn = r8 * G + rl;  // MMA N index of (row r8, head r)
+              *reinterpret_cast<uint32_t*>(mt + g * p.mt_group_stride + (nn >> 3) * 256 +
+                                           ((nn & 7) << 1)) = pack_bf16(v[r] * z, v[r + 1] * z);
+            }
+            fence_proxy_async_smem();
+          }
         }
+        tc_fence_before();
+        named_sync(kBarMt + (n & 1), 160);  // hand stage n to the MMA warp
+        vring.next();
       }
-      tc_fence_before();
-      named_sync(kBarMt + (n & 1), 160);  // hand stage n to the MMA warp
-      ++n;
     }
     // ------------------------------------------------------------ epilogue
     const int c = q * 32 + lane;  // d index = TMEM lane
@@ -452,7 +484,8 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.mt_bytes = (uint32_t(v.Hkv) * p.mt_group_stride + 127u) & ~127u;
   p.w_bytes = (uint32_t(Hr) * uint32_t(p.Hs_pad) * 2u + 127u) & ~127u;
   // deepest map ring that fits next to a V / mixed-map ring of 4 (else 3, 2)
-  const size_t budget = 227u * 1024u - 1024u - 512u - p.w_bytes;
+  const uint32_t kb_bytes = 512u * 4u;  // kept key blocks of one row (L <= 512 B)
+  const size_t budget = 227u * 1024u - 1024u - 512u - p.w_bytes - kb_bytes;
   int ms = 0, vs = 0;
   for (int cand_vs = 4; cand_vs >= 2 && ms == 0; --cand_vs) {
     const size_t fixed = size_t(cand_vs) * (p.v_bytes + p.mt_bytes);
@@ -470,7 +503,8 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.off_map = vs * p.v_bytes;
   p.off_mt = p.off_map + ms * p.map_slot;
   p.off_w = p.off_mt + vs * p.mt_bytes;
-  p.off_bar = (p.off_w + p.w_bytes + 7u) & ~7u;
+  p.off_kb = p.off_w + p.w_bytes;
+  p.off_bar = (p.off_kb + kb_bytes + 7u) & ~7u;
   const size_t smem = size_t(p.off_bar) + (2 * ms + 2 * vs + av::kMixBufs + 1) * 8 + 32 + 1024;
   const unsigned grid = unsigned(sz.nqb) * unsigned(d.B / av::kRows);
   cudaError_t e = cudaSuccess;

@@ -84,7 +84,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // phase ahead, also when a timed-out wait makes the rest of the walk a no-op.
 constexpr int kBarMt = 1;
 
+// bar.sync is warp-aligned: a warp that reaches it split (after a spin wait
+// or a one-lane branch) would be counted once per piece, so converge first.
 __device__ __forceinline__ void named_sync(int id, int count) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
@@ -258,47 +261,63 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     nst = __reduce_add_sync(0xffffffffu, nst);
     const uint32_t idesc_mix = idesc_bf16(128, HR, 1, 0);  // A MN-major, B K-major
     const uint32_t idesc_o = idesc_bf16(128, NO, 1, 1);    // A, B MN-major
-    const int ksteps = p.Hs_pad / 16;
-    const uint64_t mix_a0 = smem_desc(sbase + p.off_map, p.Hs * 128, 1024, kSwizzle128);
-    const uint64_t mix_b0 = smem_desc(sbase + p.off_w, 128, p.Hs_pad * 16, kSwizzleNone);
-    const uint64_t o_a0 = smem_desc(sbase + p.off_v, 2048, 1024, kSwizzle128);
-    const uint64_t o_b0 = smem_desc(sbase + p.off_mt, 128, 256, kSwizzleNone);
+    // Operands of tcgen05.mma live in uniform registers: derive every base
+    // from values the compiler can see are warp-uniform.
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    const uint32_t sb = __shfl_sync(0xffffffffu, sbase, 0);
+    const int ksteps = p.Hs_pad / 16;  // 1..4
+    const uint64_t mix_a0 = smem_desc(sb + p.off_map, p.Hs * 128, 1024, kSwizzle128);
+    const uint64_t mix_b0 = smem_desc(sb + p.off_w, 128, p.Hs_pad * 16, kSwizzleNone);
+    const uint64_t o_a0 = smem_desc(sb + p.off_v, 2048, 1024, kSwizzle128);
+    const uint64_t o_b0 = smem_desc(sb + p.off_mt, 128, 256, kSwizzleNone);
     const uint32_t map_step = p.map_slot >> 4, v_step = p.v_bytes >> 4,
                    mt_step = p.mt_bytes >> 4, mtg_step = p.mt_group_stride >> 4;
     Ring mring(MS), vring(VS);
-    auto issue_mix = [&](int m) {
-      const bool ok = __all_sync(0xffffffffu, wait(&map_full[mring.slot], mring.phase));
-      tc_fence_after();
-      if (ok && elect_one()) {
-        const uint64_t a = mix_a0 + uint64_t(mring.slot) * map_step;
-        const uint32_t d = tmem + kMixCol + uint32_t(m & (kMixBufs - 1)) * HR;
-        for (int kk = 0; kk < ksteps; ++kk)
+    // The elected lane alone waits and issues.  Every wait of a stage comes
+    // before any of its MMAs, and the stage's O and mix MMAs go out as one
+    // batch: an mbarrier test issued behind queued tcgen05.mma waits for them
+    // to drain, so interleaving waits with MMAs would idle the tensor pipe
+    // between batches.  The map slab arrives by bulk copy (async proxy,
+    // ordered by its mbarrier), so no tcgen05 fence sits between that wait
+    // and the MMAs.
+    auto mix_mmas = [&](int m) {
+      const uint64_t a = mix_a0 + uint64_t(mring.slot) * map_step;
+      const uint32_t d = tm + kMixCol + uint32_t(m & (kMixBufs - 1)) * HR;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        if (kk < ksteps)
           mma_bf16_ss(d, a + kk * (2048 >> 4), mix_b0 + kk * (256 >> 4), idesc_mix, kk > 0);
-        mma_commit(&map_empty[mring.slot]);
-        mma_commit(&mix_full[m & (kMixBufs - 1)]);
-      }
+      mma_commit(&map_empty[mring.slot]);
+      mma_commit(&mix_full[m & (kMixBufs - 1)]);
+    };
+    for (int m = 0; m < kMixBufs && m < nst; ++m) {
+      if (elect_one() && wait(&map_full[mring.slot], mring.phase)) mix_mmas(m);
       __syncwarp();
       mring.next();
-    };
-    for (int m = 0; m < kMixBufs && m < nst; ++m) issue_mix(m);
+    }
     for (int n = 0; n < nst; ++n) {
       named_sync(kBarMt + (n & 1), 160);  // stage n's M^T is written, its mix buffer read
-      const bool ok = __all_sync(0xffffffffu, wait(&v_full[vring.slot], vring.phase));
+      // orders the converters' TMEM reads of stage n's mix buffer before the
+      // mix MMA that overwrites it below (one fence per stage)
       tc_fence_after();
+      const bool more = n + kMixBufs < nst;
       if (elect_one()) {
-        if (ok) {
+        const bool v_ok = wait(&v_full[vring.slot], vring.phase);
+        const bool m_ok = more && wait(&map_full[mring.slot], mring.phase);
+        if (v_ok) {
           const uint64_t a = o_a0 + uint64_t(vring.slot) * v_step;
           const uint64_t b = o_b0 + uint64_t(vring.slot) * mt_step;
 #pragma unroll
           for (int g = 0; g < HKV; ++g)
-            mma_bf16_ss(tmem + g * NO, a + g * (4096 >> 4), b + uint64_t(g) * mtg_step, idesc_o,
+            mma_bf16_ss(tm + g * NO, a + g * (4096 >> 4), b + uint64_t(g) * mtg_step, idesc_o,
                         n > 0);
         }
         mma_commit(&vm_empty[vring.slot]);
+        if (m_ok) mix_mmas(n + kMixBufs);  // into the buffer stage n freed
       }
       __syncwarp();
       vring.next();
-      if (n + kMixBufs < nst) issue_mix(n + kMixBufs);  // into the buffer stage n freed
+      if (more) mring.next();
     }
     if (elect_one()) mma_commit(final_bar);
     __syncwarp();

@@ -286,6 +286,12 @@ mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int3
   return MF_OK;
 }
 
+mf_status mf_exp2_fma_eval(const float* x, float* y, int64_t n, mf_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return fail(MF_ERR_INVALID_ARG, "n < 0 or NULL array");
+  const cudaError_t e = launch_exp2_fma_eval(x, y, n, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MF_OK : cuda_fail(e, "exp2_fma_eval launch");
+}
+
 mf_status mf_sync_status(mf_stream_t stream) {
   unsigned* p = status_word();
   if (!p) return fail(MF_ERR_CUDA, "no CUDA device");

@@ -285,5 +285,54 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+// Packed pair arithmetic of sm_100 (one instruction for two f32 lanes).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x on the FMA pipe, for x <= 0 (the caller's max-subtracted logits), so
+// that part of a tile's exponentials leaves the MUFU unit free.  x = j + f
+// with j = round(x) and f in [-1/2, 1/2]: adding 1.5 * 2^23 rounds x to an
+// integer held in the low mantissa bits of t; 2^f comes from a degree-4
+// polynomial (relative minimax on [-1/2, 1/2], coefficients and their error
+// from csrc/gen_exp2_poly.py: 2.7e-6 relative with float32 Horner steps), and
+// 2^j is applied by adding j to the exponent field.  Inputs below -125 are
+// clamped so the result stays a normal float (2^-125 ~ 2.4e-38, against
+// terms of order one in every sum this feeds).
+constexpr float kExp2C0 = 0.9999992847442627f;
+constexpr float kExp2C1 = 0.6931217908859253f;
+constexpr float kExp2C2 = 0.240247443318367f;
+constexpr float kExp2C3 = 0.05591785907745361f;
+constexpr float kExp2C4 = 0.009570102207362652f;
+
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;  // 1.5 * 2^23
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(kExp2C4, f, kExp2C3);
+  p = fmaf(p, f, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 }  // namespace sm100
 }  // namespace mf

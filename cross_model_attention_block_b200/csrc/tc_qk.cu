@@ -42,6 +42,12 @@ constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB: two [128][64] swizzle
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcol = 256;  // first TMEM column of the per-key-block log partials
+// Share of the statistics exponentials computed by exp2_fma (k of every 8).
+// Measured on B200 with the 32K-token workload: 2/8 -> 7.96 ms, 3/8 -> 8.31,
+// 4/8 -> 8.89, against 7.6-8.0 ms with none: the epilogue is bound by
+// instruction issue, not by the MUFU unit, so the extra FMA-pipe instructions
+// cost more than they save.  Kept selectable; off.
+constexpr int kFmaExp = 0;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -324,15 +330,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float m_new = valid ? fmaxf(m_run, mt) : 0.f;
           // only masked keys seen so far (m = -inf): sum nothing
           const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
-          float acc[8];
+          // pairs of columns on the packed f32x2 pipe: one instruction scales
+          // and shifts two logits, one adds two exponentials
+          float2 acc[4];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+          for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+          const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m_use, -m_use);
 #pragma unroll
           for (int c = 0; c < 64; c += 8)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] += ex2(fmaf(v[c + k], sc, -m_use));
-          const float sh = ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
-                           ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+            for (int k = 0; k < 8; k += 2) {
+              const float2 x = ffma2(make_float2(v[c + k], v[c + k + 1]), sc2, nm2);
+              // kFmaExp of every 8 exponentials may run on the FMA pipe
+              const float e0 = (k >= 8 - kFmaExp) ? exp2_fma(x.x) : ex2(x.x);
+              const float e1 = (k + 1 >= 8 - kFmaExp) ? exp2_fma(x.y) : ex2(x.y);
+              acc[k >> 1] = fadd2(acc[k >> 1], make_float2(e0, e1));
+            }
+          const float sh = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                           ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
           l_run = l_run * ex2(m_run - m_use) + sh;
           m_run = m_new;
           if (BB == 64) {
@@ -373,9 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                   const int col = kgl * 16 + c * 8 + 2 * k;
-                  __nv_bfloat162 pr =
-                      __floats2bfloat162_rn(valid ? ex2(fmaf(v[col], sc, -lse2)) : 0.f,
-                                            valid ? ex2(fmaf(v[col + 1], sc, -lse2)) : 0.f);
+                  const float2 x = ffma2(make_float2(v[col], v[col + 1]), make_float2(sc, sc),
+                                         make_float2(-lse2, -lse2));
+                  __nv_bfloat162 pr = __floats2bfloat162_rn(valid ? ex2(x.x) : 0.f,
+                                                            valid ? ex2(x.y) : 0.f);
                   w4[k] = *reinterpret_cast<uint32_t*>(&pr);
                 }
                 *reinterpret_cast<uint4*>(line + (((cbase | c) ^ (h & 7)) << 4)) =
@@ -471,6 +487,13 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// y = exp2_fma(x), grid-stride (diagnostic entry point).
+__global__ void k_exp2_fma_eval(const float* __restrict__ x, float* y, int64_t n) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += int64_t(gridDim.x) * blockDim.x)
+    y[i] = exp2_fma(x[i]);
+}
 
 }  // namespace qk
 
@@ -600,6 +623,13 @@ cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const Meta
                               cudaStream_t st) {
   return launch_qk(qk::kExtract, d, sz, m, Q, K, const_cast<float*>(lse), nullptr, slot,
                    values, capacity, st);
+}
+
+cudaError_t launch_exp2_fma_eval(const float* x, float* y, int64_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 8);
+  qk::k_exp2_fma_eval<<<unsigned(blocks), 256, 0, st>>>(x, y, n);
+  return cudaGetLastError();
 }
 
 }  // namespace mf

@@ -28,7 +28,8 @@ EXPORTED = [
     "mf_block_stats", "mf_select_extract_workspace", "mf_select_extract",
     "mf_mapped_av_workspace", "mf_mapped_av", "mf_block_stats_noalloc",
     "mf_block_stats_noalloc_max_workspace",
-    "mf_sync_status", "mf_prefix_hash", "mf_index_create", "mf_index_destroy",
+    "mf_exp2_fma_eval", "mf_sync_status", "mf_prefix_hash", "mf_index_create",
+    "mf_index_destroy",
     "mf_index_insert", "mf_index_lookup", "mf_index_size",
 ]
 
@@ -85,6 +86,7 @@ def load_library(path: str = LIB_PATH):
         "mf_mapped_av": (C.c_int, [P, P, I32, P, P, P, P, SZ, P]),
         "mf_block_stats_noalloc_max_workspace": (SZ, []),
         "mf_block_stats_noalloc": (C.c_int, [P, P, P, P, P, P]),
+        "mf_exp2_fma_eval": (C.c_int, [P, P, I64, P]),
         "mf_sync_status": (C.c_int, [P]),
         "mf_prefix_hash": (C.c_int, [P, I64, I32, C.c_uint64, P]),
         "mf_index_create": (C.c_int, [P]),
@@ -274,6 +276,17 @@ def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None
                           C.c_void_p(wsp), nbytes, _stream()))
     cache._av_ws = ws  # keep the workspace alive until the stream has used it
     return O
+
+
+def exp2_fma_eval(x):
+    """2^x by the statistics kernel's FMA-pipe exponential (float32 CUDA tensor)."""
+    L = load_library()
+    if x.dtype != torch.float32 or not x.is_cuda:
+        _check(MF_ERR_INVALID_ARG)
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    _check(L.mf_exp2_fma_eval(_ptr(x), _ptr(y), x.numel(), _stream()))
+    return y
 
 
 def sync_status():

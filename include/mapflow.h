@@ -204,6 +204,16 @@ mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc,
                        int32_t Hr, const void* W, const mf_v_desc* v, void* O,
                        void* ws, size_t ws_bytes, mf_stream_t stream);
 
+/* Diagnostic, not on the hot path: y[i] = 2^x[i] by the FMA-pipe
+ * exponential that the tensor-core block-statistics kernel uses for a share
+ * of every tile's exponentials (x = j + f, j = round(x); 2^f from a degree-4
+ * polynomial with relative minimax error 2.7e-6 on [-1/2, 1/2]; 2^j added to
+ * the exponent).  Meant for x <= 0; x below -125 is clamped to -125.  x, y:
+ * device float arrays of n elements (they may be the same array).  Lets tests
+ * hold it against CUDA's exp2f.  Errors: MF_ERR_INVALID_ARG (n < 0, or a
+ * NULL array with n > 0), MF_ERR_CUDA (launch failure). */
+mf_status mf_exp2_fma_eval(const float* x, float* y, int64_t n, mf_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device status word of the
  * current device: MF_OK, MF_ERR_TIMEOUT or MF_ERR_CAPACITY. */
 mf_status mf_sync_status(mf_stream_t stream);

@@ -65,7 +65,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -332,13 +332,19 @@ def bench_ours(args, wl, rank, world, local_rank):
     stats_tf = alg["stats_flops"] / (t_stats * 1e-3) / 1e12
     ext_gbs = alg["extract_bytes"] / (t_sel * 1e-3) / 1e9
     hbm = peaks["hbm_gbs"]
-    tens = peaks["bf16_tflops"]
+    # the kernels are timed inside a loop of back-to-back steps lasting about a
+    # second, so the tensor denominator is the sustained cuBLAS figure; the
+    # fraction of the burst figure is reported beside it
+    tens = peaks["bf16_tflops_sustained"]
+    tens_burst = peaks["bf16_tflops"]
     kernels = {
         "mapped_av": {"bound": "hbm", "achieved": av_gbs, "peak": hbm, "unit": "GB/s",
                       "frac": av_gbs / hbm, "ms": t_av,
                       "algorithmic_bytes": alg["av_bytes"]},
         "block_stats": {"bound": "tensor", "achieved": stats_tf, "peak": tens,
                         "unit": "TFLOP/s", "frac": stats_tf / tens, "ms": t_stats,
+                        "peak_kind": "sustained bf16 (kernel timed inside a long step loop)",
+                        "frac_of_burst_peak": stats_tf / tens_burst,
                         "algorithmic_flops": alg["stats_flops"]},
         "select_extract": {"bound": "hbm", "achieved": ext_gbs, "peak": hbm, "unit": "GB/s",
                            "frac": ext_gbs / hbm, "ms": t_sel,
@@ -364,6 +370,7 @@ def bench_ours(args, wl, rank, world, local_rank):
         "mapped_av_gbs": av_gbs, "mapped_av_hbm_frac": av_gbs / hbm,
         "compress_tokens_per_s": wl.ntok / ((t_stats + t_sel) * 1e-3),
         "stats_tensor_frac": stats_tf / tens,
+        "stats_tensor_frac_of_burst": stats_tf / tens_burst,
         "layer_prefill_ms": t_av,
         "stage_ms": {"block_stats": t_stats, "select_extract": t_sel, "mapped_av": t_av},
         "roofline": roof, "kernels": kernels,
@@ -386,7 +393,7 @@ LAUNCHES_PER_STEP = 12
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_bf16_n32768")

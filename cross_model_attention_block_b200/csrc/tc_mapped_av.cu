@@ -66,9 +66,11 @@ struct Params {
   int64_t capacity;
   int64_t nqb;
   int Hs, Hs_pad, Hr, Hkv, G, B;
-  uint32_t map_bytes;       // Hs * 256 (one stage)
-  uint32_t map_slot;        // map_bytes + 1 KB zero guard, 1 KB aligned
-  uint32_t v_bytes, mt_group_stride, mt_bytes, w_bytes;
+  uint32_t map_bytes;       // Hs * 256: one 16-key group's slab
+  uint32_t map_slot;        // KG slabs + 1 KB guard, 1 KB aligned
+  uint32_t v_bytes;         // 4096 * Hkv: one 16-key group's V image
+  uint32_t v_slot;          // KG images
+  uint32_t mt_group_stride, mt_bytes, w_bytes;
   uint32_t off_v, off_map, off_mt, off_w, off_kb, off_bar;
   int map_stages, vm_stages;
   unsigned* status;
@@ -114,19 +116,41 @@ struct Ring {
   }
 };
 
-// A stage is (kept entry e, 16-key group kg) of the CTA's query block; key
-// groups that start past the sequence end are skipped.
+// 16-key groups of key block kb that hold keys of the sequence.
 __device__ __forceinline__ int key_groups_of(int kb, int B, int L) {
   const int rem = L - kb * B;
   return rem <= 0 ? 0 : min(B, rem + kKeys - 1) / kKeys;
 }
 
-template <int HR, int G>
+// A stage is up to KG consecutive 16-key groups of one kept entry of the
+// CTA's query block (the last stage of an entry may hold fewer); every role
+// walks the same list, read from the kept-block list in shared memory.
+template <int KG>
+struct Stages {
+  const int32_t* kb_list;
+  int nE, B, L;
+  int e = -1, kb = 0, kg0 = 0, nkg = 0;
+  __device__ Stages(const int32_t* list, int n, int b, int l) : kb_list(list), nE(n), B(b), L(l) {}
+  __device__ bool next() {
+    kg0 += KG;
+    while (kg0 >= nkg) {
+      if (++e >= nE) return false;
+      kb = kb_list[e];
+      nkg = key_groups_of(kb, B, L);
+      kg0 = 0;
+    }
+    return true;
+  }
+  __device__ int nk() const { return min(KG, nkg - kg0); }  // groups in this stage
+};
+
+template <int HR, int G, int KG>
 __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   constexpr int HKV = HR / G;
   constexpr int NO = kRows * G;          // O MMA N per group
   constexpr uint32_t kMixCol = 8u * HR;  // first TMEM column of the mix accumulators
-  static_assert(kMixCol + kMixBufs * HR <= kTmemCols, "O^T and mix accumulators exceed TMEM");
+  constexpr uint32_t kMixCols = KG * HR;  // one stage's mix accumulator (KG M-tiles)
+  static_assert(kMixCol + kMixBufs * kMixCols <= kTmemCols, "O^T and mix accumulators exceed TMEM");
   static_assert((kMixBufs & (kMixBufs - 1)) == 0, "kMixBufs must be a power of two");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -175,8 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   }
   // W^T as the K-major operand [Hr rows][Hs_pad], core matrices of 8 rows x 16
   // bytes, K chunks 128 bytes apart, row groups Hs_pad * 16 bytes apart; zero
-  // past Hs.  The 1 KB guard after every map slot is zeroed (the padded K
-  // step of the mix reads it).
+  // past Hs.  The map ring is zeroed: the padded K step of the mix reads past
+  // a slab (into the next slab or the 1 KB guard), where it must meet finite
+  // values for the zero rows of W^T to cancel them.
   {
     uint8_t* wt = base + p.off_w;
     for (int idx = threadIdx.x; idx < HR * p.Hs_pad; idx += kThreads) {
@@ -185,10 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
       *reinterpret_cast<__nv_bfloat16*>(wt + (r >> 3) * (p.Hs_pad * 16) + (h >> 3) * 128 +
                                         (r & 7) * 16 + (h & 7) * 2) = w;
     }
-    for (int st = 0; st < MS; ++st) {
-      uint32_t* g = reinterpret_cast<uint32_t*>(base + p.off_map + st * p.map_slot + p.map_bytes);
-      for (int k = threadIdx.x; k < 256; k += kThreads) g[k] = 0u;
-    }
+    uint4* ring = reinterpret_cast<uint4*>(base + p.off_map);
+    for (uint32_t k = threadIdx.x; k < uint32_t(MS) * p.map_slot / 16u; k += kThreads)
+      ring[k] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -197,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(base);
-  const int S8 = p.B / 8;
+  const int S8 = p.B / 8, S16 = p.B / kKeys;
   // a wait that gave up makes every later wait of the CTA give up at once, so
   // the named-barrier hand-offs below still run to the end without blocking
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -211,43 +235,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     // ------------------------------------------------------- map producer
     if (lane == 0) {
       Ring ring(MS);
-      bool live = true;
-      for (int e = 0; e < nE && live; ++e) {
-        const int nk = key_groups_of(s_kb[e], p.B, L);
-        const int64_t line_e = (e0 + e) * (p.B / 16);
-        for (int kg = 0; kg < nk; ++kg) {
-          if (!wait(&map_empty[ring.slot], ring.phase ^ 1u)) {
-            live = false;
-            break;
-          }
-          mbar_expect_tx(&map_full[ring.slot], p.map_bytes);
-          const int64_t line0 = ((line_e + kg) * S8 + slice) * 2 * p.Hs;
-          bulk_load(base + p.off_map + ring.slot * p.map_slot, p.values + line0 * 64,
-                    p.map_bytes, &map_full[ring.slot]);
-          ring.next();
+      Stages<KG> st(s_kb, nE, p.B, L);
+      while (st.next()) {
+        if (!wait(&map_empty[ring.slot], ring.phase ^ 1u)) break;
+        const int nk = st.nk();
+        mbar_expect_tx(&map_full[ring.slot], uint32_t(nk) * p.map_bytes);
+        for (int h = 0; h < nk; ++h) {
+          const int64_t line0 = (((e0 + st.e) * S16 + st.kg0 + h) * S8 + slice) * 2 * p.Hs;
+          bulk_load(base + p.off_map + ring.slot * p.map_slot + h * p.map_bytes,
+                    p.values + line0 * 64, p.map_bytes, &map_full[ring.slot]);
         }
+        ring.next();
       }
     }
   } else if (warp == 2) {
     // --------------------------------------------------------- V producer
     if (lane == 0) {
       Ring ring(VS);
+      Stages<KG> st(s_kb, nE, p.B, L);
       const int64_t g0 = p.cu_g[s];
-      bool live = true;
-      for (int e = 0; e < nE && live; ++e) {
-        const int kb = s_kb[e];
-        const int nk = key_groups_of(kb, p.B, L);
-        for (int kg = 0; kg < nk; ++kg) {
-          if (!wait(&vm_empty[ring.slot], ring.phase ^ 1u)) {
-            live = false;
-            break;
-          }
-          mbar_expect_tx(&v_full[ring.slot], p.v_bytes);
-          const int64_t grp = g0 + int64_t(kb) * (p.B / kKeys) + kg;
-          bulk_load(base + p.off_v + ring.slot * p.v_bytes, p.vimg + grp * p.v_bytes, p.v_bytes,
-                    &v_full[ring.slot]);
-          ring.next();
-        }
+      while (st.next()) {
+        if (!wait(&vm_empty[ring.slot], ring.phase ^ 1u)) break;
+        const uint32_t bytes = uint32_t(st.nk()) * p.v_bytes;  // consecutive images
+        mbar_expect_tx(&v_full[ring.slot], bytes);
+        const int64_t grp = g0 + int64_t(st.kb) * S16 + st.kg0;
+        bulk_load(base + p.off_v + ring.slot * p.v_slot, p.vimg + grp * p.v_bytes, bytes,
+                  &v_full[ring.slot]);
+        ring.next();
       }
     }
   } else if (warp == 1) {
@@ -257,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     // start-address field moves (added in 16-byte units, never carrying out
     // of its 14 bits), and ring positions advance without division.
     int nst = 0;
-    for (int e = lane; e < nE; e += 32) nst += key_groups_of(s_kb[e], p.B, L);
+    for (int e = lane; e < nE; e += 32) nst += (key_groups_of(s_kb[e], p.B, L) + KG - 1) / KG;
     nst = __reduce_add_sync(0xffffffffu, nst);
     const uint32_t idesc_mix = idesc_bf16(128, HR, 1, 0);  // A MN-major, B K-major
     const uint32_t idesc_o = idesc_bf16(128, NO, 1, 1);    // A, B MN-major
@@ -269,10 +283,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     const uint64_t mix_a0 = smem_desc(sb + p.off_map, p.Hs * 128, 1024, kSwizzle128);
     const uint64_t mix_b0 = smem_desc(sb + p.off_w, 128, p.Hs_pad * 16, kSwizzleNone);
     const uint64_t o_a0 = smem_desc(sb + p.off_v, 2048, 1024, kSwizzle128);
-    const uint64_t o_b0 = smem_desc(sb + p.off_mt, 128, 256, kSwizzleNone);
-    const uint32_t map_step = p.map_slot >> 4, v_step = p.v_bytes >> 4,
-                   mt_step = p.mt_bytes >> 4, mtg_step = p.mt_group_stride >> 4;
+    const uint64_t o_b0 = smem_desc(sb + p.off_mt, 128, KG * 256, kSwizzleNone);
+    const uint32_t map_step = p.map_slot >> 4, map_half = p.map_bytes >> 4,
+                   v_step = p.v_slot >> 4, v_half = p.v_bytes >> 4, mt_step = p.mt_bytes >> 4,
+                   mtg_step = p.mt_group_stride >> 4;
     Ring mring(MS), vring(VS);
+    Stages<KG> cur(s_kb, nE, p.B, L), ahead(s_kb, nE, p.B, L);
     // The elected lane alone waits and issues.  Every wait of a stage comes
     // before any of its MMAs, and the stage's O and mix MMAs go out as one
     // batch: an mbarrier test issued behind queued tcgen05.mma waits for them
@@ -280,40 +296,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     // between batches.  The map slab arrives by bulk copy (async proxy,
     // ordered by its mbarrier), so no tcgen05 fence sits between that wait
     // and the MMAs.
-    auto mix_mmas = [&](int m) {
+    auto mix_mmas = [&](int m, int nk) {
       const uint64_t a = mix_a0 + uint64_t(mring.slot) * map_step;
-      const uint32_t d = tm + kMixCol + uint32_t(m & (kMixBufs - 1)) * HR;
+      const uint32_t d = tm + kMixCol + uint32_t(m & (kMixBufs - 1)) * kMixCols;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        if (kk < ksteps)
-          mma_bf16_ss(d, a + kk * (2048 >> 4), mix_b0 + kk * (256 >> 4), idesc_mix, kk > 0);
+      for (int h = 0; h < KG; ++h)
+        if (h < nk)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            if (kk < ksteps)
+              mma_bf16_ss(d + h * HR, a + h * map_half + kk * (2048 >> 4),
+                          mix_b0 + kk * (256 >> 4), idesc_mix, kk > 0);
       mma_commit(&map_empty[mring.slot]);
       mma_commit(&mix_full[m & (kMixBufs - 1)]);
     };
     for (int m = 0; m < kMixBufs && m < nst; ++m) {
-      if (elect_one() && wait(&map_full[mring.slot], mring.phase)) mix_mmas(m);
+      ahead.next();
+      if (elect_one() && wait(&map_full[mring.slot], mring.phase)) mix_mmas(m, ahead.nk());
       __syncwarp();
       mring.next();
     }
     for (int n = 0; n < nst; ++n) {
+      cur.next();
+      const bool more = n + kMixBufs < nst;
+      if (more) ahead.next();
       named_sync(kBarMt + (n & 1), 160);  // stage n's M^T is written, its mix buffer read
       // orders the converters' TMEM reads of stage n's mix buffer before the
       // mix MMA that overwrites it below (one fence per stage)
       tc_fence_after();
-      const bool more = n + kMixBufs < nst;
       if (elect_one()) {
         const bool v_ok = wait(&v_full[vring.slot], vring.phase);
         const bool m_ok = more && wait(&map_full[mring.slot], mring.phase);
         if (v_ok) {
           const uint64_t a = o_a0 + uint64_t(vring.slot) * v_step;
           const uint64_t b = o_b0 + uint64_t(vring.slot) * mt_step;
+          const int nk = cur.nk();
 #pragma unroll
-          for (int g = 0; g < HKV; ++g)
-            mma_bf16_ss(tm + g * NO, a + g * (4096 >> 4), b + uint64_t(g) * mtg_step, idesc_o,
-                        n > 0);
+          for (int h = 0; h < KG; ++h)
+            if (h < nk)
+#pragma unroll
+              for (int g = 0; g < HKV; ++g)
+                mma_bf16_ss(tm + g * NO, a + h * v_half + g * (4096 >> 4),
+                            b + uint64_t(g) * mtg_step + h * (256 >> 4), idesc_o, n > 0 || h > 0);
         }
         mma_commit(&vm_empty[vring.slot]);
-        if (m_ok) mix_mmas(n + kMixBufs);  // into the buffer stage n freed
+        if (m_ok) mix_mmas(n + kMixBufs, ahead.nk());  // into the buffer stage n freed
       }
       __syncwarp();
       vring.next();
@@ -323,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ converters
-    // One thread per mix-accumulator lane = (row, key) pair.
+    // One thread per mix-accumulator lane = (row, key) pair of each M-tile.
     const int q = warp & 3;  // TMEM lane quarter: pairs 32q .. 32q+31
     const int m = q * 32 + lane;
     const int r8 = m >> 4, k16 = m & 15;
@@ -331,39 +358,44 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
     const bool row_ok = i0 + r8 < L;
     uint8_t* mt0 = base + p.off_mt + (k16 >> 3) * 128 + (k16 & 7) * 16;
     Ring vring(VS);
+    Stages<KG> st(s_kb, nE, p.B, L);
     int n = 0;
-    for (int e = 0; e < nE; ++e) {
-      const int kb = s_kb[e];
-      const int nk = key_groups_of(kb, p.B, L);
-      for (int kg = 0; kg < nk; ++kg, ++n) {
-        const int db = n & (kMixBufs - 1);
-        if (wait(&mix_full[db], uint32_t(n / kMixBufs) & 1u)) {
-          tc_fence_after();
-          float v[HR];
-          if constexpr (HR == 32) {
-            tmem_ld32(lane_addr + kMixCol + db * HR, v);
-          } else {
-            tmem_ld16(lane_addr + kMixCol + db * HR, v);
-          }
-          tmem_wait_ld();
-          if (wait(&vm_empty[vring.slot], vring.phase ^ 1u)) {  // M^T slot free
-            const int key = kb * p.B + kg * kKeys + k16;
-            const float z = (key < L && row_ok) ? 1.f : 0.f;
-            uint8_t* mt = mt0 + vring.slot * p.mt_bytes;
+    while (st.next()) {
+      const int db = n & (kMixBufs - 1);
+      if (wait(&mix_full[db], uint32_t(n / kMixBufs) & 1u)) {
+        tc_fence_after();
+        if (wait(&vm_empty[vring.slot], vring.phase ^ 1u)) {  // M^T slot free
+          const int nk = st.nk();
+          uint8_t* mt = mt0 + vring.slot * p.mt_bytes;
 #pragma unroll
-            for (int r = 0; r < HR; r += 2) {
-              const int g = r / G, rl = r % G;
-              const int nn = r8 * G + rl;  // MMA N index of (row r8, head r)
-              *reinterpret_cast<uint32_t*>(mt + g * p.mt_group_stride + (nn >> 3) * 256 +
-                                           ((nn & 7) << 1)) = pack_bf16(v[r] * z, v[r + 1] * z);
+          for (int h = 0; h < KG; ++h) {
+            if (h < nk) {
+              float v[HR];
+              if constexpr (HR == 32) {
+                tmem_ld32(lane_addr + kMixCol + db * kMixCols + h * HR, v);
+              } else {
+                tmem_ld16(lane_addr + kMixCol + db * kMixCols + h * HR, v);
+              }
+              tmem_wait_ld();
+              const int key = st.kb * p.B + (st.kg0 + h) * kKeys + k16;
+              const bool keep = key < L && row_ok;  // select, never multiply stale values
+#pragma unroll
+              for (int r = 0; r < HR; r += 2) {
+                const int g = r / G, rl = r % G;
+                const int nn = r8 * G + rl;  // MMA N index of (row r8, head r)
+                *reinterpret_cast<uint32_t*>(mt + h * 256 + g * p.mt_group_stride +
+                                             (nn >> 3) * (KG * 256) + ((nn & 7) << 1)) =
+                    keep ? pack_bf16(v[r], v[r + 1]) : 0u;
+              }
             }
-            fence_proxy_async_smem();
           }
+          fence_proxy_async_smem();
         }
-        tc_fence_before();
-        named_sync(kBarMt + (n & 1), 160);  // hand stage n to the MMA warp
-        vring.next();
       }
+      tc_fence_before();
+      named_sync(kBarMt + (n & 1), 160);  // hand stage n to the MMA warp
+      vring.next();
+      ++n;
     }
     // ------------------------------------------------------------ epilogue
     const int c = q * 32 + lane;  // d index = TMEM lane
@@ -497,29 +529,39 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.B = d.B;
   p.status = status_word();
   p.map_bytes = 256u * uint32_t(d.Hs);
-  p.map_slot = (p.map_bytes + 1024u + 1023u) & ~1023u;
   p.v_bytes = 4096u * uint32_t(v.Hkv);
-  p.mt_group_stride = 256u * uint32_t(p.G) + 16u;
-  p.mt_bytes = (uint32_t(v.Hkv) * p.mt_group_stride + 127u) & ~127u;
   p.w_bytes = (uint32_t(Hr) * uint32_t(p.Hs_pad) * 2u + 127u) & ~127u;
-  // deepest map ring that fits next to a V / mixed-map ring of 4 (else 3, 2)
   const uint32_t kb_bytes = 512u * 4u;  // kept key blocks of one row (L <= 512 B)
   const size_t budget = 227u * 1024u - 1024u - 512u - p.w_bytes - kb_bytes;
-  int ms = 0, vs = 0;
-  for (int cand_vs = 4; cand_vs >= 2 && ms == 0; --cand_vs) {
-    const size_t fixed = size_t(cand_vs) * (p.v_bytes + p.mt_bytes);
-    for (int cand_ms = av::kMaxMapStages; cand_ms >= 2; --cand_ms)
-      if (fixed + size_t(cand_ms) * p.map_slot <= budget) {
-        ms = cand_ms;
-        vs = cand_vs;
-        break;
-      }
+  // Stages of 32 keys (two 16-key groups) when two V / M^T slots and two map
+  // slots fit: half the per-stage waits, commits and hand-offs of 16-key
+  // stages.  Otherwise 16-key stages with the deepest rings that fit.
+  int kg = 0, ms = 0, vs = 0;
+  for (int cand_kg = 2; cand_kg >= 1 && ms == 0; --cand_kg) {
+    const uint32_t map_slot = (uint32_t(cand_kg) * p.map_bytes + 1024u + 1023u) & ~1023u;
+    const uint32_t mtg = uint32_t(cand_kg) * 256u * uint32_t(p.G) + 16u;
+    const uint32_t mt_bytes = (uint32_t(v.Hkv) * mtg + 127u) & ~127u;
+    const uint32_t v_slot = uint32_t(cand_kg) * p.v_bytes;
+    for (int cand_vs = (cand_kg == 2 ? 2 : 4); cand_vs >= 2 && ms == 0; --cand_vs) {
+      const size_t fixed = size_t(cand_vs) * (v_slot + mt_bytes);
+      for (int cand_ms = av::kMaxMapStages; cand_ms >= 2; --cand_ms)
+        if (fixed + size_t(cand_ms) * map_slot <= budget) {
+          kg = cand_kg;
+          ms = cand_ms;
+          vs = cand_vs;
+          p.map_slot = map_slot;
+          p.mt_group_stride = mtg;
+          p.mt_bytes = mt_bytes;
+          p.v_slot = v_slot;
+          break;
+        }
+    }
   }
   if (ms == 0) return cudaErrorInvalidConfiguration;
   p.map_stages = ms;
   p.vm_stages = vs;
   p.off_v = 0;
-  p.off_map = vs * p.v_bytes;
+  p.off_map = vs * p.v_slot;
   p.off_mt = p.off_map + ms * p.map_slot;
   p.off_w = p.off_mt + vs * p.mt_bytes;
   p.off_kb = p.off_w + p.w_bytes;
@@ -527,18 +569,23 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   const size_t smem = size_t(p.off_bar) + (2 * ms + 2 * vs + av::kMixBufs + 1) * 8 + 32 + 1024;
   const unsigned grid = unsigned(sz.nqb) * unsigned(d.B / av::kRows);
   cudaError_t e = cudaSuccess;
-#define MF_AV(HR, G)                                                                        \
+#define MF_AV(HR, G, KG)                                                                    \
   do {                                                                                      \
-    e = cudaFuncSetAttribute(av::k_mapped_av<HR, G>,                                        \
+    e = cudaFuncSetAttribute(av::k_mapped_av<HR, G, KG>,                                    \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));       \
     if (e != cudaSuccess) return e;                                                         \
-    av::k_mapped_av<HR, G><<<grid, av::kThreads, smem, st>>>(p);                            \
+    av::k_mapped_av<HR, G, KG><<<grid, av::kThreads, smem, st>>>(p);                        \
+  } while (0)
+#define MF_AV_G(HR, KG)                                                                     \
+  do {                                                                                      \
+    if (p.G == 2) MF_AV(HR, 2, KG); else if (p.G == 4) MF_AV(HR, 4, KG); else MF_AV(HR, 8, KG); \
   } while (0)
   if (Hr == 32) {
-    if (p.G == 2) MF_AV(32, 2); else if (p.G == 4) MF_AV(32, 4); else MF_AV(32, 8);
+    if (kg == 2) MF_AV_G(32, 2); else MF_AV_G(32, 1);
   } else {
-    if (p.G == 2) MF_AV(16, 2); else if (p.G == 4) MF_AV(16, 4); else MF_AV(16, 8);
+    if (kg == 2) MF_AV_G(16, 2); else MF_AV_G(16, 1);
   }
+#undef MF_AV_G
 #undef MF_AV
   return cudaGetLastError();
 }

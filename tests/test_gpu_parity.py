@@ -172,7 +172,12 @@ def test_varlen_paged_workload_sampled():
     dict(lengths=[390], Hs=40, Hr=32, Hkv=8, B=128, tau=0.9),
     dict(lengths=[257, 31], Hs=32, Hr=16, Hkv=4, B=64, tau=0.8),
     dict(lengths=[160], Hs=16, Hr=16, Hkv=8, B=128, tau=0.95),
-], ids=["hs40_b64", "hs40_b128", "hs32_g4_b64", "hs16_g2_b128"])
+    # 16-key stages: V images of 16 KV heads, or 64 sender heads, leave no
+    # room for two 32-key stages in shared memory
+    dict(lengths=[270], Hs=40, Hr=32, Hkv=16, B=64, tau=0.9),
+    dict(lengths=[200, 77], Hs=64, Hr=32, Hkv=8, B=128, tau=0.9),
+], ids=["hs40_b64", "hs40_b128", "hs32_g4_b64", "hs16_g2_b128", "hs40_kv16_b64_16key",
+        "hs64_b128_16key"])
 def test_mapped_av_on_an_oracle_built_cache(case):
     """The fused kernel alone: cache (CSR + probability blocks) written from the
     oracle, O compared with the oracle's."""

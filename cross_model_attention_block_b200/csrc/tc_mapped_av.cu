@@ -45,7 +45,7 @@ namespace av {
 constexpr int kRows = 8;   // query rows per CTA
 constexpr int kKeys = 16;  // keys per stage
 constexpr int kD = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // warps 0-3 roles, 4-11 converters (two per lane quarter)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxMapStages = 8;
 // Mix accumulators in TMEM: mix(n + kMixBufs) is issued as soon as stage n has
@@ -85,6 +85,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // to the MMA warp: both sides bar.sync once per stage, so neither can run a
 // phase ahead, also when a timed-out wait makes the rest of the walk a no-op.
 constexpr int kBarMt = 1;
+constexpr int kConverterWarps = 8;
+constexpr int kHandOff = kConverterWarps * 32 + 32;  // named-barrier count: converters + O warp
 
 // bar.sync is warp-aligned: a warp that reaches it split (after a spin wait
 // or a one-lane branch) would be counted once per piece, so converge first.
@@ -161,7 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   uint64_t* v_full = map_empty + MS;                                    // [VS]
   uint64_t* vm_empty = v_full + VS;                                     // [VS]
   uint64_t* mix_full = vm_empty + VS;                                   // [kMixBufs]
-  uint64_t* final_bar = mix_full + kMixBufs;
+  uint64_t* mix_empty = mix_full + kMixBufs;                            // [kMixBufs]
+  uint64_t* final_bar = mix_empty + kMixBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_kb = reinterpret_cast<int32_t*>(base + p.off_kb);  // kept key blocks of the row
@@ -192,7 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
       mbar_init(&v_full[i], 1);
       mbar_init(&vm_empty[i], 1);
     }
-    for (int i = 0; i < kMixBufs; ++i) mbar_init(&mix_full[i], 1);
+    for (int i = 0; i < kMixBufs; ++i) {
+      mbar_init(&mix_full[i], 1);
+      mbar_init(&mix_empty[i], kConverterWarps);
+    }
     mbar_init(final_bar, 1);
     *abort = 0;
     fence_barrier_init();
@@ -264,99 +270,106 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
         ring.next();
       }
     }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------- MMA warp
-    // The whole warp walks the stages (it takes part in the named barriers);
-    // one elected lane issues.  Descriptors are built once, per MMA only the
-    // start-address field moves (added in 16-byte units, never carrying out
-    // of its 14 bits), and ring positions advance without division.
-    int nst = 0;
-    for (int e = lane; e < nE; e += 32) nst += (key_groups_of(s_kb[e], p.B, L) + KG - 1) / KG;
-    nst = __reduce_add_sync(0xffffffffu, nst);
-    const uint32_t idesc_mix = idesc_bf16(128, HR, 1, 0);  // A MN-major, B K-major
-    const uint32_t idesc_o = idesc_bf16(128, NO, 1, 1);    // A, B MN-major
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------- O warp / mix warp
+    // Two issuing warps with disjoint accumulators: warp 1 issues the O
+    // products (accumulating O^T), warp 3 the head mix (into the four mix
+    // buffers), each from one elected lane while the warp walks the stages
+    // converged.  Descriptors are built once, per MMA only the start-address
+    // field moves (added in 16-byte units, never carrying out of its 14
+    // bits), and ring positions advance without division.  The mix warp runs
+    // up to kMixBufs stages ahead, gated by the map slab and by the
+    // converters releasing the buffer; the O warp takes each stage from the
+    // converters through the named barrier.
     // Operands of tcgen05.mma live in uniform registers: derive every base
     // from values the compiler can see are warp-uniform.
     const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
     const uint32_t sb = __shfl_sync(0xffffffffu, sbase, 0);
-    const int ksteps = p.Hs_pad / 16;  // 1..4
-    const uint64_t mix_a0 = smem_desc(sb + p.off_map, p.Hs * 128, 1024, kSwizzle128);
-    const uint64_t mix_b0 = smem_desc(sb + p.off_w, 128, p.Hs_pad * 16, kSwizzleNone);
-    const uint64_t o_a0 = smem_desc(sb + p.off_v, 2048, 1024, kSwizzle128);
-    const uint64_t o_b0 = smem_desc(sb + p.off_mt, 128, KG * 256, kSwizzleNone);
-    const uint32_t map_step = p.map_slot >> 4, map_half = p.map_bytes >> 4,
-                   v_step = p.v_slot >> 4, v_half = p.v_bytes >> 4, mt_step = p.mt_bytes >> 4,
-                   mtg_step = p.mt_group_stride >> 4;
-    Ring mring(MS), vring(VS);
-    Stages<KG> cur(s_kb, nE, p.B, L), ahead(s_kb, nE, p.B, L);
-    // The elected lane alone waits and issues.  Every wait of a stage comes
-    // before any of its MMAs, and the stage's O and mix MMAs go out as one
-    // batch: an mbarrier test issued behind queued tcgen05.mma waits for them
-    // to drain, so interleaving waits with MMAs would idle the tensor pipe
-    // between batches.  The map slab arrives by bulk copy (async proxy,
-    // ordered by its mbarrier), so no tcgen05 fence sits between that wait
-    // and the MMAs.
-    auto mix_mmas = [&](int m, int nk) {
-      const uint64_t a = mix_a0 + uint64_t(mring.slot) * map_step;
-      const uint32_t d = tm + kMixCol + uint32_t(m & (kMixBufs - 1)) * kMixCols;
+    Stages<KG> st(s_kb, nE, p.B, L);
+    if (warp == 3) {
+      const uint32_t idesc_mix = idesc_bf16(128, HR, 1, 0);  // A MN-major, B K-major
+      const int ksteps = p.Hs_pad / 16;                     // 1..4
+      const uint64_t mix_a0 = smem_desc(sb + p.off_map, p.Hs * 128, 1024, kSwizzle128);
+      const uint64_t mix_b0 = smem_desc(sb + p.off_w, 128, p.Hs_pad * 16, kSwizzleNone);
+      const uint32_t map_step = p.map_slot >> 4, map_half = p.map_bytes >> 4;
+      Ring mring(MS);
+      int m = 0;
+      while (st.next()) {
+        const int db = m & (kMixBufs - 1);
+        if (elect_one()) {
+          // the map slab arrives by bulk copy (async proxy, ordered by its
+          // mbarrier); the converters' TMEM reads of the buffer's previous
+          // stage are ordered by mix_empty and the fence
+          const bool ok = wait(&map_full[mring.slot], mring.phase) &&
+                          wait(&mix_empty[db], (uint32_t(m / kMixBufs) & 1u) ^ 1u);
+          tc_fence_after();
+          if (ok) {
+            const uint64_t a = mix_a0 + uint64_t(mring.slot) * map_step;
+            const uint32_t d = tm + kMixCol + uint32_t(db) * kMixCols;
+            const int nk = st.nk();
 #pragma unroll
-      for (int h = 0; h < KG; ++h)
-        if (h < nk)
+            for (int h = 0; h < KG; ++h)
+              if (h < nk)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            if (kk < ksteps)
-              mma_bf16_ss(d + h * HR, a + h * map_half + kk * (2048 >> 4),
-                          mix_b0 + kk * (256 >> 4), idesc_mix, kk > 0);
-      mma_commit(&map_empty[mring.slot]);
-      mma_commit(&mix_full[m & (kMixBufs - 1)]);
-    };
-    for (int m = 0; m < kMixBufs && m < nst; ++m) {
-      ahead.next();
-      if (elect_one() && wait(&map_full[mring.slot], mring.phase)) mix_mmas(m, ahead.nk());
-      __syncwarp();
-      mring.next();
-    }
-    for (int n = 0; n < nst; ++n) {
-      cur.next();
-      const bool more = n + kMixBufs < nst;
-      if (more) ahead.next();
-      named_sync(kBarMt + (n & 1), 160);  // stage n's M^T is written, its mix buffer read
-      // orders the converters' TMEM reads of stage n's mix buffer before the
-      // mix MMA that overwrites it below (one fence per stage)
-      tc_fence_after();
-      if (elect_one()) {
-        const bool v_ok = wait(&v_full[vring.slot], vring.phase);
-        const bool m_ok = more && wait(&map_full[mring.slot], mring.phase);
-        if (v_ok) {
-          const uint64_t a = o_a0 + uint64_t(vring.slot) * v_step;
-          const uint64_t b = o_b0 + uint64_t(vring.slot) * mt_step;
-          const int nk = cur.nk();
-#pragma unroll
-          for (int h = 0; h < KG; ++h)
-            if (h < nk)
-#pragma unroll
-              for (int g = 0; g < HKV; ++g)
-                mma_bf16_ss(tm + g * NO, a + h * v_half + g * (4096 >> 4),
-                            b + uint64_t(g) * mtg_step + h * (256 >> 4), idesc_o, n > 0 || h > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                  if (kk < ksteps)
+                    mma_bf16_ss(d + h * HR, a + h * map_half + kk * (2048 >> 4),
+                                mix_b0 + kk * (256 >> 4), idesc_mix, kk > 0);
+            mma_commit(&map_empty[mring.slot]);
+            mma_commit(&mix_full[db]);
+          }
         }
-        mma_commit(&vm_empty[vring.slot]);
-        if (m_ok) mix_mmas(n + kMixBufs, ahead.nk());  // into the buffer stage n freed
+        __syncwarp();
+        mring.next();
+        ++m;
       }
+    } else {
+      const uint32_t idesc_o = idesc_bf16(128, NO, 1, 1);  // A, B MN-major
+      const uint64_t o_a0 = smem_desc(sb + p.off_v, 2048, 1024, kSwizzle128);
+      const uint64_t o_b0 = smem_desc(sb + p.off_mt, 128, KG * 256, kSwizzleNone);
+      const uint32_t v_step = p.v_slot >> 4, v_half = p.v_bytes >> 4,
+                     mt_step = p.mt_bytes >> 4, mtg_step = p.mt_group_stride >> 4;
+      Ring vring(VS);
+      int n = 0;
+      while (st.next()) {
+        named_sync(kBarMt + (n & 1), kHandOff);  // stage n's M^T is written
+        tc_fence_after();
+        if (elect_one()) {
+          if (wait(&v_full[vring.slot], vring.phase)) {
+            const uint64_t a = o_a0 + uint64_t(vring.slot) * v_step;
+            const uint64_t b = o_b0 + uint64_t(vring.slot) * mt_step;
+            const int nk = st.nk();
+#pragma unroll
+            for (int h = 0; h < KG; ++h)
+              if (h < nk)
+#pragma unroll
+                for (int g = 0; g < HKV; ++g)
+                  mma_bf16_ss(tm + g * NO, a + h * v_half + g * (4096 >> 4),
+                              b + uint64_t(g) * mtg_step + h * (256 >> 4), idesc_o,
+                              n > 0 || h > 0);
+          }
+          mma_commit(&vm_empty[vring.slot]);
+        }
+        __syncwarp();
+        vring.next();
+        ++n;
+      }
+      if (elect_one()) mma_commit(final_bar);
       __syncwarp();
-      vring.next();
-      if (more) mring.next();
     }
-    if (elect_one()) mma_commit(final_bar);
-    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ converters
-    // One thread per mix-accumulator lane = (row, key) pair of each M-tile.
-    const int q = warp & 3;  // TMEM lane quarter: pairs 32q .. 32q+31
+    // One thread per mix-accumulator lane = (row, key) pair of each M-tile;
+    // the two warps of a lane quarter split the receiver heads (columns).
+    constexpr int HH = HR / 2;  // heads per converter warp
+    const int q = warp & 3;     // TMEM lane quarter: pairs 32q .. 32q+31
+    const int hh = (warp - 4) >> 2;
     const int m = q * 32 + lane;
     const int r8 = m >> 4, k16 = m & 15;
     const uint32_t lane_addr = tmem + (uint32_t(q * 32) << 16);
     const bool row_ok = i0 + r8 < L;
-    uint8_t* mt0 = base + p.off_mt + (k16 >> 3) * 128 + (k16 & 7) * 16;
+    uint8_t* mt0 = base + p.off_mt + (k16 >> 3) * 128 + (k16 & 7) * 16 +
+                   (hh * (HH / G)) * p.mt_group_stride;
     Ring vring(VS);
     Stages<KG> st(s_kb, nE, p.B, L);
     int n = 0;
@@ -370,19 +383,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
 #pragma unroll
           for (int h = 0; h < KG; ++h) {
             if (h < nk) {
-              float v[HR];
-              if constexpr (HR == 32) {
-                tmem_ld32(lane_addr + kMixCol + db * kMixCols + h * HR, v);
+              float v[HH];
+              const uint32_t col = lane_addr + kMixCol + db * kMixCols + h * HR + hh * HH;
+              if constexpr (HH == 16) {
+                tmem_ld16(col, v);
               } else {
-                tmem_ld16(lane_addr + kMixCol + db * kMixCols + h * HR, v);
+                tmem_ld8(col, v);
               }
               tmem_wait_ld();
+              if (h + 1 == nk) {  // the stage's mix buffer is read: release it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&mix_empty[db]);
+              }
               const int key = st.kb * p.B + (st.kg0 + h) * kKeys + k16;
               const bool keep = key < L && row_ok;  // select, never multiply stale values
 #pragma unroll
-              for (int r = 0; r < HR; r += 2) {
-                const int g = r / G, rl = r % G;
-                const int nn = r8 * G + rl;  // MMA N index of (row r8, head r)
+              for (int r = 0; r < HH; r += 2) {
+                const int g = r / G, rl = r % G;  // group relative to this warp's first
+                const int nn = r8 * G + rl;       // MMA N index of (row r8, head)
                 *reinterpret_cast<uint32_t*>(mt + h * 256 + g * p.mt_group_stride +
                                              (nn >> 3) * (KG * 256) + ((nn & 7) << 1)) =
                     keep ? pack_bf16(v[r], v[r + 1]) : 0u;
@@ -393,16 +412,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
         }
       }
       tc_fence_before();
-      named_sync(kBarMt + (n & 1), 160);  // hand stage n to the MMA warp
+      named_sync(kBarMt + (n & 1), kHandOff);  // hand stage n to the O warp
       vring.next();
       ++n;
     }
     // ------------------------------------------------------------ epilogue
-    const int c = q * 32 + lane;  // d index = TMEM lane
+    // O^T of the GQA groups g with g % 2 == hh (TMEM lane = d), stored to O.
+    const int c = q * 32 + lane;  // d index
     const bool ok = wait(final_bar, 0);
     tc_fence_after();
 #pragma unroll 1
-    for (int g = 0; g < HKV; ++g) {
+    for (int g = hh; g < HKV; g += 2) {
 #pragma unroll
       for (int c0 = 0; c0 < NO; c0 += 16) {
         float o[16];
@@ -566,7 +586,7 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.off_w = p.off_mt + vs * p.mt_bytes;
   p.off_kb = p.off_w + p.w_bytes;
   p.off_bar = (p.off_kb + kb_bytes + 7u) & ~7u;
-  const size_t smem = size_t(p.off_bar) + (2 * ms + 2 * vs + av::kMixBufs + 1) * 8 + 32 + 1024;
+  const size_t smem = size_t(p.off_bar) + (2 * ms + 2 * vs + 2 * av::kMixBufs + 1) * 8 + 32 + 1024;
   const unsigned grid = unsigned(sz.nqb) * unsigned(d.B / av::kRows);
   cudaError_t e = cudaSuccess;
 #define MF_AV(HR, G, KG)                                                                    \

@@ -160,9 +160,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
   const int MS = p.map_stages, VS = p.vm_stages;
   uint64_t* map_full = reinterpret_cast<uint64_t*>(base + p.off_bar);  // [MS]
   uint64_t* map_empty = map_full + MS;                                  // [MS]
-  uint64_t* v_full = map_empty + MS;                                    // [VS]
-  uint64_t* vm_empty = v_full + VS;                                     // [VS]
-  uint64_t* mix_full = vm_empty + VS;                                   // [kMixBufs]
+  // V ring: one barrier pair per 16-key half of a slot, so a half is refilled
+  // as soon as the O products that read it are done
+  uint64_t* v_full = map_empty + MS;                                    // [VS][KG]
+  uint64_t* vm_empty = v_full + VS * KG;                                // [VS][KG]
+  uint64_t* mix_full = vm_empty + VS * KG;                              // [kMixBufs]
   uint64_t* mix_empty = mix_full + kMixBufs;                            // [kMixBufs]
   uint64_t* final_bar = mix_empty + kMixBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
       mbar_init(&map_full[i], 1);
       mbar_init(&map_empty[i], 1);
     }
-    for (int i = 0; i < VS; ++i) {
+    for (int i = 0; i < VS * KG; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&vm_empty[i], 1);
     }
@@ -260,13 +262,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
       Ring ring(VS);
       Stages<KG> st(s_kb, nE, p.B, L);
       const int64_t g0 = p.cu_g[s];
-      while (st.next()) {
-        if (!wait(&vm_empty[ring.slot], ring.phase ^ 1u)) break;
-        const uint32_t bytes = uint32_t(st.nk()) * p.v_bytes;  // consecutive images
-        mbar_expect_tx(&v_full[ring.slot], bytes);
+      bool live = true;
+      while (live && st.next()) {
+        const int nk = st.nk();
         const int64_t grp = g0 + int64_t(st.kb) * S16 + st.kg0;
-        bulk_load(base + p.off_v + ring.slot * p.v_slot, p.vimg + grp * p.v_bytes, bytes,
-                  &v_full[ring.slot]);
+        for (int h = 0; h < KG; ++h) {
+          uint64_t* full = &v_full[ring.slot * KG + h];
+          if (!wait(&vm_empty[ring.slot * KG + h], ring.phase ^ 1u)) {
+            live = false;
+            break;
+          }
+          // a half past the stage's groups still completes its phase (no bytes)
+          mbar_expect_tx(full, h < nk ? p.v_bytes : 0u);
+          if (h < nk)
+            bulk_load(base + p.off_v + ring.slot * p.v_slot + h * p.v_bytes,
+                      p.vimg + (grp + h) * p.v_bytes, p.v_bytes, full);
+        }
         ring.next();
       }
     }
@@ -335,20 +346,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
         named_sync(kBarMt + (n & 1), kHandOff);  // stage n's M^T is written
         tc_fence_after();
         if (elect_one()) {
-          if (wait(&v_full[vring.slot], vring.phase)) {
-            const uint64_t a = o_a0 + uint64_t(vring.slot) * v_step;
-            const uint64_t b = o_b0 + uint64_t(vring.slot) * mt_step;
-            const int nk = st.nk();
+          const uint64_t a = o_a0 + uint64_t(vring.slot) * v_step;
+          const uint64_t b = o_b0 + uint64_t(vring.slot) * mt_step;
+          const int nk = st.nk();
 #pragma unroll
-            for (int h = 0; h < KG; ++h)
-              if (h < nk)
+          for (int h = 0; h < KG; ++h) {
+            // each half of the V slot is waited for, consumed and released on
+            // its own; a half past the stage's groups only passes its phase
+            if (wait(&v_full[vring.slot * KG + h], vring.phase) && h < nk) {
 #pragma unroll
-                for (int g = 0; g < HKV; ++g)
-                  mma_bf16_ss(tm + g * NO, a + h * v_half + g * (4096 >> 4),
-                              b + uint64_t(g) * mtg_step + h * (256 >> 4), idesc_o,
-                              n > 0 || h > 0);
+              for (int g = 0; g < HKV; ++g)
+                mma_bf16_ss(tm + g * NO, a + h * v_half + g * (4096 >> 4),
+                            b + uint64_t(g) * mtg_step + h * (256 >> 4), idesc_o,
+                            n > 0 || h > 0);
+            }
+            mma_commit(&vm_empty[vring.slot * KG + h]);
           }
-          mma_commit(&vm_empty[vring.slot]);
         }
         __syncwarp();
         vring.next();
@@ -377,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
       const int db = n & (kMixBufs - 1);
       if (wait(&mix_full[db], uint32_t(n / kMixBufs) & 1u)) {
         tc_fence_after();
-        if (wait(&vm_empty[vring.slot], vring.phase ^ 1u)) {  // M^T slot free
+        // the M^T slot is free once all of O(n - VS) is done: its last half's commit
+        if (wait(&vm_empty[vring.slot * KG + KG - 1], vring.phase ^ 1u)) {
           const int nk = st.nk();
           uint8_t* mt = mt0 + vring.slot * p.mt_bytes;
 #pragma unroll
@@ -586,7 +600,8 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.off_w = p.off_mt + vs * p.mt_bytes;
   p.off_kb = p.off_w + p.w_bytes;
   p.off_bar = (p.off_kb + kb_bytes + 7u) & ~7u;
-  const size_t smem = size_t(p.off_bar) + (2 * ms + 2 * vs + 2 * av::kMixBufs + 1) * 8 + 32 + 1024;
+  const size_t smem =
+      size_t(p.off_bar) + (2 * ms + 2 * vs * kg + 2 * av::kMixBufs + 1) * 8 + 32 + 1024;
   const unsigned grid = unsigned(sz.nqb) * unsigned(d.B / av::kRows);
   cudaError_t e = cudaSuccess;
 #define MF_AV(HR, G, KG)                                                                    \

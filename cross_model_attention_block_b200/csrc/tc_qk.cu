@@ -37,6 +37,7 @@ namespace qk {
 constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kStages = 3;
+constexpr int kMaxBlocksPerSeq = 512;  // a sequence holds at most 512 blocks
 constexpr int kThreads = 384;  // warps 0-3 roles, 4-11 epilogue (two per lane quarter)
 constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB: two [128][64] swizzled halves
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
@@ -61,6 +62,10 @@ struct Smem {
   uint8_t out[2][kTileBytes];
   float red[2][4][32];
   float2 xch[4][64];  // per-row (max, sum) exchange between the two warpgroups
+  // extraction: cache entry of (row block a of this query tile, key block kb),
+  // -1 where the block is not kept or not causal; read by every role instead
+  // of the global block -> entry map
+  int32_t slots[2][kMaxBlocksPerSeq];
   uint64_t q_full;
   uint64_t k_full[kStages];
   uint64_t k_empty[kStages];
@@ -90,24 +95,15 @@ struct Params {
   unsigned* status;
 };
 
-// Does key tile kt of query tile t hold a kept block (extract) -- every
-// causal key tile counts for the statistics.
+// Does key tile kt hold a kept block of this query tile (extract) -- every
+// causal key tile counts for the statistics.  `slots` is the CTA's copy of
+// the block -> entry map (-1: not kept or not causal).
 template <int MODE, int BB>
-__device__ __forceinline__ bool tile_needed(const Params& p, int s, int t, int kt, int nqb_s) {
+__device__ __forceinline__ bool tile_needed(const int32_t (*slots)[kMaxBlocksPerSeq], int kt) {
   if (MODE == kStats) return true;
-  const int64_t cb = p.cu_blk[s];
-  if (BB == 128) {
-    return p.slot[cb + int64_t(t) * (t + 1) / 2 + kt] >= 0;
-  }
-  for (int a = 0; a < 2; ++a) {
-    int qb = 2 * t + a;
-    if (qb >= nqb_s) break;
-    for (int b = 0; b < 2; ++b) {
-      int kb = 2 * kt + b;
-      if (kb <= qb && p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kb] >= 0) return true;
-    }
-  }
-  return false;
+  if (BB == 128) return slots[0][kt] >= 0;
+  return slots[0][2 * kt] >= 0 || slots[0][2 * kt + 1] >= 0 || slots[1][2 * kt] >= 0 ||
+         slots[1][2 * kt + 1] >= 0;
 }
 
 // Lane l ends up holding sum over the warp of v[l] (v has 32 entries).
@@ -196,6 +192,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
+  if (MODE == kExtract) {
+    const int64_t cb = p.cu_blk[s];
+    for (int i = threadIdx.x; i < 2 * kMaxBlocksPerSeq; i += kThreads) {
+      const int a = i / kMaxBlocksPerSeq, kb = i % kMaxBlocksPerSeq;
+      const int qb = (BB == 128) ? (a == 0 ? t : -1) : 2 * t + a;
+      sm.slots[a][kb] = (qb >= 0 && qb < nqb_s && kb <= qb)
+                            ? p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kb]
+                            : -1;
+    }
+  }
   if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -212,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(sm.q + kHalfBytes, &tmQ, &sm.q_full, h * kD + 64, seq0 + row0);
       int n = 0;
       for (int kt = 0; kt <= t; ++kt) {
-        if (!tile_needed<MODE, BB>(p, s, t, kt, nqb_s)) continue;
+        if (!tile_needed<MODE, BB>(sm.slots, kt)) continue;
         const int st = n % kStages;
         if (!mbar_wait(&sm.k_empty[st], ((n / kStages) & 1) ^ 1, p.status)) break;
         mbar_expect_tx(&sm.k_full[st], kTileBytes);
@@ -230,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&sm.q_full, 0, p.status);
       int n = 0;
       for (int kt = 0; ok && kt <= t; ++kt) {
-        if (!tile_needed<MODE, BB>(p, s, t, kt, nqb_s)) continue;
+        if (!tile_needed<MODE, BB>(sm.slots, kt)) continue;
         const int st = n % kStages, sb = n & 1;
         if (!mbar_wait(&sm.k_full[st], (n / kStages) & 1, p.status)) break;
         if (!mbar_wait(&sm.s_empty[sb], ((n >> 1) & 1) ^ 1, p.status)) break;
@@ -268,12 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -CUDART_INF_F, l_run = 0.f;  // this group's online max and sum
     float lse2 = 0.f;
     if (MODE == kExtract) lse2 = valid ? p.lse[int64_t(h) * p.ntok + seq0 + ri] * kLog2e : 0.f;
-    const int qb_r = (BB == 128) ? t : 2 * t + (r >> 6);
     const int64_t cb = p.cu_blk[s];
     int n = 0;
     bool ok = true;
     for (int kt = 0; kt <= t; ++kt) {
-      if (!tile_needed<MODE, BB>(p, s, t, kt, nqb_s)) continue;
+      if (!tile_needed<MODE, BB>(sm.slots, kt)) continue;
       if ((n & 1) != wg) { ++n; continue; }
       const int sb = wg;
       bool got = mbar_wait(&sm.s_full[sb], (n >> 1) & 1, p.status);
@@ -375,8 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int lrow = ((rb >> 3) << 1) + ((rb & 7) >> 2);  // line of this row, key group 0
           const int cbase = (rb & 3) << 1;                       // chunk of keys 0-7
           const int kb = (BB == 128) ? kt : 2 * kt + ch;
-          if (qb_r < nqb_s && kb <= qb_r &&
-              p.slot[cb + int64_t(qb_r) * (qb_r + 1) / 2 + kb] >= 0) {
+          if (sm.slots[(BB == 128) ? 0 : (r >> 6)][kb] >= 0) {  // kept (so causal, row exists)
             uint8_t* sub = obuf + ((BB == 128) ? 0 : ((r >> 6) * 2 + ch) * 8192);
 #pragma unroll
             for (int kgl = 0; kgl < 4; ++kgl) {
@@ -407,13 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
 #pragma unroll
           for (int a = 0; a < kTile / BB; ++a) {
-            const int qb = (BB == 128) ? t : 2 * t + a;
-            if (qb >= nqb_s) continue;
 #pragma unroll
             for (int b = 0; b < kTile / BB; ++b) {
               const int kbb = kt * (kTile / BB) + b;
-              if (kbb > qb) continue;
-              const int64_t e = p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kbb];
+              const int e = sm.slots[a][kbb];  // -1: not kept, not causal or no such row block
               if (e < 0) continue;
               const uint8_t* sub = obuf + ((BB == 128) ? 0 : (a * 2 + b) * 8192);
               tma_store_4d(&tmV, sub, 0, h, 0, int32_t(e));

@@ -228,6 +228,21 @@ def algorithmic(wl, nnz):
                 av_flops=av_flops, map_bytes=map_bytes)
 
 
+def max_over_ranks(x, world, device):
+    """The largest value of x over all ranks (every rank gets it); x itself at N=1."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process if unset)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
 def bench_ours(args, wl, rank, world, local_rank):
     from cross_model_attention_block_b200 import mapflow as mfb
 
@@ -282,10 +297,7 @@ def bench_ours(args, wl, rank, world, local_rank):
     ms = t_start.elapsed_time(t_end)
     stage = np.array([[m[i].elapsed_time(m[i + 1]) for i in range(3)] for m in marks])
     stage_ms = stage.mean(axis=0)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     mfb.sync_status()
 
     # end to end through the C ABI: host inputs in, host output back
@@ -313,11 +325,7 @@ def bench_ours(args, wl, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     mfb.sync_status()
     h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hW))
     d2h = hO.numel() * hO.element_size()
@@ -390,7 +398,7 @@ def bench_ours(args, wl, rank, world, local_rank):
 LAUNCHES_PER_STEP = 12
 
 
-def main():
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
@@ -398,11 +406,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_bf16_n32768")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     wl = synth.workloads()[args.workload]
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = rank_env()
     if args.impl == "reference":
         if rank == 0:
             bench_reference(args, wl)

@@ -1,0 +1,68 @@
+"""The N > 1 host path of bench.py with two gloo ranks on CPU: rank
+environment, the max-over-ranks timing reduction every rank takes part in,
+and the reference arm that runs on rank 0 only."""
+import os
+import socket
+import sys
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        r, w, lr = bench.rank_env()
+        # per-rank "timed region" lengths; every rank must see the slowest
+        got = bench.max_over_ranks(10.0 + 5.0 * rank, w, torch.device("cpu"))
+        got2 = bench.max_over_ranks(7.0 - rank, w, torch.device("cpu"))
+        dist.barrier()
+        out[rank] = (r, w, lr, got, got2)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_with_two_gloo_ranks():
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0] == (0, 2, 0, 15.0, 7.0)
+    assert res[1] == (1, 2, 1, 15.0, 7.0)
+
+
+def test_single_process_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    """Under torchrun every rank but 0 exits 0 without work and prints nothing."""
+    sys.path.insert(0, ROOT)
+    import bench
+    called = []
+    monkeypatch.setattr(bench, "bench_reference", lambda args, wl: called.append(wl.name))
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--gpus", "2"]) == 0
+    assert called == [] and capsys.readouterr().out == ""
+    monkeypatch.setenv("RANK", "0")
+    assert bench.main(["--impl", "reference", "--gpus", "2"]) == 0
+    assert called == ["large_bf16_n32768"]

@@ -292,6 +292,13 @@ mf_status mf_exp2_fma_eval(const float* x, float* y, int64_t n, mf_stream_t stre
   return e == cudaSuccess ? MF_OK : cuda_fail(e, "exp2_fma_eval launch");
 }
 
+mf_status mf_selftest_timeout(int32_t limit_ms, mf_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return fail(MF_ERR_INVALID_ARG, "limit_ms must be in [1, 2000]");
+  const cudaError_t e =
+      launch_selftest_timeout(uint64_t(limit_ms) * 1000000ull, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MF_OK : cuda_fail(e, "selftest_timeout launch");
+}
+
 mf_status mf_sync_status(mf_stream_t stream) {
   unsigned* p = status_word();
   if (!p) return fail(MF_ERR_CUDA, "no CUDA device");

@@ -77,6 +77,7 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
                                 int64_t key_groups, cudaStream_t st);
 
 cudaError_t launch_exp2_fma_eval(const float* x, float* y, int64_t n, cudaStream_t st);
+cudaError_t launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
                               const void* Q, const void* K, float* lse, float* part,
                               cudaStream_t st);

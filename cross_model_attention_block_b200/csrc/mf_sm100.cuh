@@ -74,17 +74,22 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Wait for the phase with the given parity to complete; false after kWaitNs
 // (the status word then carries kStatusTimeout).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned* status,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     for (int k = 0; k < 8; ++k)
       if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-    if (global_ns() - t0 > kWaitNs) {
+    if (global_ns() - t0 > limit_ns) {
       atomicOr(status, kStatusTimeout);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status) {
+  return mbar_wait_for(bar, parity, status, kWaitNs);
 }
 
 // ------------------------------------------------------------------------ TMA

@@ -489,6 +489,17 @@ using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, 
                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// One thread waits, with the kernels' bounded wait, on an mbarrier whose
+// phase nothing completes: the wait gives up after limit_ns and raises the
+// timeout bit of the status word (diagnostic entry point for the failure path).
+__global__ void k_selftest_timeout(uint64_t limit_ns, unsigned* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  mbar_wait_for(&bar, 0, status, limit_ns);  // expected to return false
+}
+
 // y = exp2_fma(x), grid-stride (diagnostic entry point).
 __global__ void k_exp2_fma_eval(const float* __restrict__ x, float* y, int64_t n) {
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -630,6 +641,11 @@ cudaError_t launch_exp2_fma_eval(const float* x, float* y, int64_t n, cudaStream
   if (n == 0) return cudaSuccess;
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 8);
   qk::k_exp2_fma_eval<<<unsigned(blocks), 256, 0, st>>>(x, y, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st) {
+  qk::k_selftest_timeout<<<1, 32, 0, st>>>(limit_ns, status_word());
   return cudaGetLastError();
 }
 

@@ -28,7 +28,8 @@ EXPORTED = [
     "mf_block_stats", "mf_select_extract_workspace", "mf_select_extract",
     "mf_mapped_av_workspace", "mf_mapped_av", "mf_block_stats_noalloc",
     "mf_block_stats_noalloc_max_workspace",
-    "mf_exp2_fma_eval", "mf_sync_status", "mf_prefix_hash", "mf_index_create",
+    "mf_exp2_fma_eval", "mf_selftest_timeout", "mf_sync_status", "mf_prefix_hash",
+    "mf_index_create",
     "mf_index_destroy",
     "mf_index_insert", "mf_index_lookup", "mf_index_size",
 ]
@@ -87,6 +88,7 @@ def load_library(path: str = LIB_PATH):
         "mf_block_stats_noalloc_max_workspace": (SZ, []),
         "mf_block_stats_noalloc": (C.c_int, [P, P, P, P, P, P]),
         "mf_exp2_fma_eval": (C.c_int, [P, P, I64, P]),
+        "mf_selftest_timeout": (C.c_int, [I32, P]),
         "mf_sync_status": (C.c_int, [P]),
         "mf_prefix_hash": (C.c_int, [P, I64, I32, C.c_uint64, P]),
         "mf_index_create": (C.c_int, [P]),
@@ -287,6 +289,11 @@ def exp2_fma_eval(x):
     y = torch.empty_like(x)
     _check(L.mf_exp2_fma_eval(_ptr(x), _ptr(y), x.numel(), _stream()))
     return y
+
+
+def selftest_timeout(limit_ms=20):
+    """Make one bounded device wait give up (nothing completes its barrier)."""
+    _check(load_library().mf_selftest_timeout(int(limit_ms), _stream()))
 
 
 def sync_status():

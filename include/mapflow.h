@@ -214,6 +214,14 @@ mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc,
  * NULL array with n > 0), MF_ERR_CUDA (launch failure). */
 mf_status mf_exp2_fma_eval(const float* x, float* y, int64_t n, mf_stream_t stream);
 
+/* Diagnostic, for tests of the failure path: launches one kernel whose
+ * bounded wait (the same one every tensor-core kernel uses) waits on an
+ * mbarrier phase that nothing completes, gives up after limit_ms and raises
+ * the timeout bit of the device status word, so the next mf_sync_status
+ * returns MF_ERR_TIMEOUT.  Nothing faults; the context stays usable.
+ * limit_ms in [1, 2000].  Errors: MF_ERR_INVALID_ARG, MF_ERR_CUDA. */
+mf_status mf_selftest_timeout(int32_t limit_ms, mf_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device status word of the
  * current device: MF_OK, MF_ERR_TIMEOUT or MF_ERR_CAPACITY. */
 mf_status mf_sync_status(mf_stream_t stream);

@@ -182,3 +182,8 @@ def test_index_same_key_newest_wins(lib):
     cache, seq, matched = ix.lookup(h, 0)
     assert (cache.values, seq, matched) == (15, 1, 4)
     assert len(ix) == 4
+
+
+def test_selftest_timeout_rejects_bad_limits(lib):
+    assert lib.mf_selftest_timeout(0, None) == mfb.MF_ERR_INVALID_ARG
+    assert lib.mf_selftest_timeout(5000, None) == mfb.MF_ERR_INVALID_ARG

@@ -228,6 +228,36 @@ def algorithmic(wl, nnz):
                 av_flops=av_flops, map_bytes=map_bytes)
 
 
+def dense_attention_ms(wl, dev, stream, ev, warmup, steps):
+    """Mean time of torch's causal SDPA for the receiver layer (Hr query heads,
+    Hkv KV heads, d) over the workload's sequences; a library call, reported
+    beside the fused kernel as context, never on our path."""
+    import torch.nn.functional as F
+    g = torch.Generator(device=dev).manual_seed(7)
+    dt = wl.torch_dtype
+    seqs = []
+    for L in wl.lengths:
+        q = torch.randn(1, wl.Hr, L, wl.d, device=dev, dtype=dt, generator=g)
+        k = torch.randn(1, wl.Hkv, L, wl.d, device=dev, dtype=dt, generator=g)
+        v = torch.randn(1, wl.Hkv, L, wl.d, device=dev, dtype=dt, generator=g)
+        seqs.append((q, k, v))
+
+    def run():
+        for q, k, v in seqs:
+            F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(steps):
+        run()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
 def max_over_ranks(x, world, device):
     """The largest value of x over all ranks (every rank gets it); x itself at N=1."""
     if world <= 1:
@@ -299,6 +329,12 @@ def bench_ours(args, wl, rank, world, local_rank):
     stage_ms = stage.mean(axis=0)
     ms = max_over_ranks(ms, world, dev)
     mfb.sync_status()
+
+    # context only: dense causal GQA attention of the same receiver layer
+    # (torch scaled_dot_product_attention, bf16, per sequence), the cost the
+    # fused kernel stands in for
+    dense_ms = dense_attention_ms(wl, dev, stream, ev, args.warmup, min(args.steps, 10))
+    dense_ms = max_over_ranks(dense_ms, world, dev)
 
     # end to end through the C ABI: host inputs in, host output back
     pin = lambda t: t.pin_memory()  # noqa: E731
@@ -380,6 +416,7 @@ def bench_ours(args, wl, rank, world, local_rank):
         "stats_tensor_frac": stats_tf / tens,
         "stats_tensor_frac_of_burst": stats_tf / tens_burst,
         "layer_prefill_ms": t_av,
+        "dense_sdpa_ms_context": dense_ms,
         "stage_ms": {"block_stats": t_stats, "select_extract": t_sel, "mapped_av": t_av},
         "roofline": roof, "kernels": kernels,
         "clocks": clk,

@@ -268,11 +268,21 @@ size_t mf_mapped_av_workspace(const mf_csr_cache* cache, const mf_attn_desc* des
 mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int32_t Hr,
                        const void* W, const mf_v_desc* v, void* O, void* ws, size_t ws_bytes,
                        mf_stream_t stream) {
+  if (!cache) return fail(MF_ERR_INVALID_ARG, "cache is NULL");
+  return mf_mapped_av_range(cache, desc, Hr, W, v, O, 0, cache->nqb_total, ws, ws_bytes,
+                            stream);
+}
+
+mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc, int32_t Hr,
+                             const void* W, const mf_v_desc* v, void* O, int64_t qb_begin,
+                             int64_t qb_end, void* ws, size_t ws_bytes, mf_stream_t stream) {
   Sizes sz;
   mf_status st = check_av(cache, desc, Hr, v, &sz);
   if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
   if (!W || !O) return fail(MF_ERR_INVALID_ARG, "W or O is NULL");
+  if (qb_begin < 0 || qb_begin > qb_end || qb_end > sz.nqb)
+    return fail(MF_ERR_INVALID_ARG, "query-block range outside [0, nqb_total]");
   const bool tc = mapped_av_tc_supported(d, Hr, *v);
   if (tc && (!ws || !aligned256(ws) ||
              ws_bytes < mapped_av_tc_workspace(d.nseq, key_groups(d), v->Hkv)))
@@ -280,8 +290,9 @@ mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int3
   if (!status_word()) return fail(MF_ERR_CUDA, "no CUDA device");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (sz.nqb == 0) return MF_OK;
-  cudaError_t e = tc ? launch_mapped_av_tc(*cache, d, sz, Hr, W, *v, O, ws, key_groups(d), s)
-                     : launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, s);
+  cudaError_t e = tc ? launch_mapped_av_tc(*cache, d, sz, Hr, W, *v, O, ws, key_groups(d),
+                                           qb_begin, qb_end, s)
+                     : launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, qb_begin, qb_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "mapped av");
   return MF_OK;
 }

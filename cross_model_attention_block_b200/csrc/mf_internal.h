@@ -72,9 +72,11 @@ bool mapped_av_tc_supported(const mf_attn_desc& d, int Hr, const mf_v_desc& v);
 // Workspace of the tensor-core fused kernel: per-sequence 16-key-group prefix
 // sums and V regrouped per 16 keys into operand images (4096 * Hkv bytes each).
 size_t mapped_av_tc_workspace(int nseq, int64_t key_groups, int Hkv);
+// Both fused-kernel launchers cover the global query blocks [qb_lo, qb_hi).
 cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, const Sizes& sz,
                                 int Hr, const void* W, const mf_v_desc& v, void* O, void* ws,
-                                int64_t key_groups, cudaStream_t st);
+                                int64_t key_groups, int64_t qb_lo, int64_t qb_hi,
+                                cudaStream_t st);
 
 cudaError_t launch_exp2_fma_eval(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
@@ -94,6 +96,7 @@ cudaError_t launch_extract_simt(const mf_attn_desc& d, const Sizes& sz, const vo
 
 cudaError_t launch_mapped_av_simt(const mf_csr_cache& c, const mf_attn_desc& d,
                                   const Sizes& sz, int Hr, const void* W,
-                                  const mf_v_desc& v, void* O, cudaStream_t st);
+                                  const mf_v_desc& v, void* O, int64_t qb_lo, int64_t qb_hi,
+                                  cudaStream_t st);
 
 }  // namespace mf

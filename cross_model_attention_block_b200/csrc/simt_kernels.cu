@@ -281,12 +281,13 @@ __global__ void __launch_bounds__(kAvThreads) k_mapped_av_simt(
     const int32_t* __restrict__ col_idx, int64_t capacity, const int32_t* __restrict__ qb_seq,
     const int32_t* __restrict__ qb_idx, const int32_t* __restrict__ cu_seqlens,
     const T* __restrict__ W, const T* __restrict__ V, const int32_t* __restrict__ page_table,
-    int page_size, int max_pages, int Hs, int Hr, int Hkv, int d, int B,
+    int page_size, int max_pages, int Hs, int Hr, int Hkv, int d, int B, int64_t qb_lo,
     T* __restrict__ O) {
   extern __shared__ float sm[];
   float* Ws = sm;             // [Hr][Hs]
   float* Ms = sm + Hr * Hs;   // [Hr][kAvKeys]
-  const int gqb = blockIdx.x, il = blockIdx.y, tid = threadIdx.x;
+  const int64_t gqb = qb_lo + blockIdx.x;
+  const int il = blockIdx.y, tid = threadIdx.x;
   const int s = qb_seq[gqb], qb = qb_idx[gqb];
   const int seq0 = cu_seqlens[s];
   const int L = cu_seqlens[s + 1] - seq0;
@@ -336,15 +337,17 @@ __global__ void __launch_bounds__(kAvThreads) k_mapped_av_simt(
 
 cudaError_t launch_mapped_av_simt(const mf_csr_cache& c, const mf_attn_desc& d,
                                   const Sizes& sz, int Hr, const void* W,
-                                  const mf_v_desc& v, void* O, cudaStream_t st) {
-  dim3 grid(unsigned(c.nqb_total), unsigned(d.B));
+                                  const mf_v_desc& v, void* O, int64_t qb_lo, int64_t qb_hi,
+                                  cudaStream_t st) {
+  if (qb_hi <= qb_lo) return cudaSuccess;
+  dim3 grid(unsigned(qb_hi - qb_lo), unsigned(d.B));
   size_t smem = sizeof(float) * (size_t(Hr) * d.Hs + size_t(Hr) * kAvKeys);
 #define MF_AV(T)                                                                        \
   k_mapped_av_simt<T><<<grid, kAvThreads, smem, st>>>(                                  \
       static_cast<const T*>(c.values), c.row_ptr, c.col_idx, c.nnz_capacity, c.qb_seq,   \
       c.qb_idx,                                                                         \
       d.cu_seqlens, static_cast<const T*>(W), static_cast<const T*>(v.V), v.page_table, \
-      v.page_size, v.max_pages_per_seq, d.Hs, Hr, v.Hkv, v.d, d.B, static_cast<T*>(O))
+      v.page_size, v.max_pages_per_seq, d.Hs, Hr, v.Hkv, v.d, d.B, qb_lo, static_cast<T*>(O))
   if (d.dt == MF_F32) MF_AV(float); else MF_AV(__nv_bfloat16);
 #undef MF_AV
   return cudaGetLastError();

@@ -64,7 +64,7 @@ struct Params {
   const __nv_bfloat16* W;     // [Hr][Hs]
   __nv_bfloat16* O;           // [ntok][Hr][d]
   int64_t capacity;
-  int64_t nqb;
+  int64_t qb_hi;  // CTAs cover the global query blocks [qb_hi - grid / slices, qb_hi)
   int Hs, Hs_pad, Hr, Hkv, G, B;
   uint32_t map_bytes;       // Hs * 256: one 16-key group's slab
   uint32_t map_slot;        // KG slabs + 1 KB guard, 1 KB aligned
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mapped_av(const Params p) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slices = p.B / kRows;
-  const int64_t gqb = p.nqb - 1 - blockIdx.x / slices;  // longest rows first
+  const int64_t gqb = p.qb_hi - 1 - blockIdx.x / slices;  // longest rows first
   const int slice = blockIdx.x % slices;
   const int s = p.qb_seq[gqb], qb = p.qb_idx[gqb];
   const int seq0 = p.cu_seqlens[s];
@@ -530,8 +530,9 @@ size_t mapped_av_tc_workspace(int nseq, int64_t key_groups, int Hkv) {
 
 cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, const Sizes& sz,
                                 int Hr, const void* W, const mf_v_desc& v, void* O, void* ws,
-                                int64_t key_groups, cudaStream_t st) {
-  if (c.nnz_capacity < 1 || sz.nqb == 0 || key_groups == 0) return cudaSuccess;
+                                int64_t key_groups, int64_t qb_lo, int64_t qb_hi,
+                                cudaStream_t st) {
+  if (c.nnz_capacity < 1 || qb_hi <= qb_lo || key_groups == 0) return cudaSuccess;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int32_t* cu_g = reinterpret_cast<int32_t*>(wsb);
   const size_t meta = (size_t(d.nseq + 1) * 4 + 255) & ~size_t(255);
@@ -554,7 +555,7 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.W = static_cast<const __nv_bfloat16*>(W);
   p.O = static_cast<__nv_bfloat16*>(O);
   p.capacity = c.nnz_capacity;
-  p.nqb = sz.nqb;
+  p.qb_hi = qb_hi;
   p.Hs = d.Hs;
   p.Hs_pad = (d.Hs + 15) / 16 * 16;
   p.Hr = Hr;
@@ -602,7 +603,7 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.off_bar = (p.off_kb + kb_bytes + 7u) & ~7u;
   const size_t smem =
       size_t(p.off_bar) + (2 * ms + 2 * vs * kg + 2 * av::kMixBufs + 1) * 8 + 32 + 1024;
-  const unsigned grid = unsigned(sz.nqb) * unsigned(d.B / av::kRows);
+  const unsigned grid = unsigned(qb_hi - qb_lo) * unsigned(d.B / av::kRows);
   cudaError_t e = cudaSuccess;
 #define MF_AV(HR, G, KG)                                                                    \
   do {                                                                                      \

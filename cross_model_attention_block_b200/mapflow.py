@@ -26,7 +26,7 @@ MF_BF16, MF_F32 = 0, 1
 EXPORTED = [
     "mf_version", "mf_last_error", "mf_layout_sizes", "mf_block_stats_workspace",
     "mf_block_stats", "mf_select_extract_workspace", "mf_select_extract",
-    "mf_mapped_av_workspace", "mf_mapped_av", "mf_block_stats_noalloc",
+    "mf_mapped_av_workspace", "mf_mapped_av", "mf_mapped_av_range", "mf_block_stats_noalloc",
     "mf_block_stats_noalloc_max_workspace",
     "mf_exp2_fma_eval", "mf_selftest_timeout", "mf_sync_status", "mf_prefix_hash",
     "mf_index_create",
@@ -85,6 +85,7 @@ def load_library(path: str = LIB_PATH):
         "mf_select_extract": (C.c_int, [P, P, P, P, P, C.c_double, P, P, SZ, P]),
         "mf_mapped_av_workspace": (SZ, [P, P, I32, P]),
         "mf_mapped_av": (C.c_int, [P, P, I32, P, P, P, P, SZ, P]),
+        "mf_mapped_av_range": (C.c_int, [P, P, I32, P, P, P, I64, I64, P, SZ, P]),
         "mf_block_stats_noalloc_max_workspace": (SZ, []),
         "mf_block_stats_noalloc": (C.c_int, [P, P, P, P, P, P]),
         "mf_exp2_fma_eval": (C.c_int, [P, P, I64, P]),
@@ -251,11 +252,13 @@ def select_extract(ctx: Context, Q, K, lse, mass, tau, cache: Cache | None = Non
 
 
 def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None,
-              workspace=None):
+              workspace=None, qb_range=None):
     """Stage 3: O [ntok, Hr, d] = (W-mixed kept map) x V (fused).
 
     `workspace` may be a uint8 device tensor reused across calls (grown when
-    too small); by default one is allocated per call."""
+    too small); by default one is allocated per call.  `qb_range` =
+    (begin, end) restricts the call to those global query blocks (chunked
+    prefill, prefix reuse): only their rows of O are written."""
     L = load_library()
     ctx = cache.ctx
     d = ctx.desc()
@@ -274,8 +277,13 @@ def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None
         wsp = ws.data_ptr() + (-ws.data_ptr()) % 256
     else:
         ws, wsp = _workspace(nbytes, W.device)
-    _check(L.mf_mapped_av(C.byref(cs), C.byref(d), int(Hr), _ptr(W), C.byref(vd), _ptr(O),
-                          C.c_void_p(wsp), nbytes, _stream()))
+    if qb_range is None:
+        _check(L.mf_mapped_av(C.byref(cs), C.byref(d), int(Hr), _ptr(W), C.byref(vd), _ptr(O),
+                              C.c_void_p(wsp), nbytes, _stream()))
+    else:
+        _check(L.mf_mapped_av_range(C.byref(cs), C.byref(d), int(Hr), _ptr(W), C.byref(vd),
+                                    _ptr(O), int(qb_range[0]), int(qb_range[1]),
+                                    C.c_void_p(wsp), nbytes, _stream()))
     cache._av_ws = ws  # keep the workspace alive until the stream has used it
     return O
 

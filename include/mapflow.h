@@ -204,6 +204,24 @@ mf_status mf_mapped_av(const mf_csr_cache* cache, const mf_attn_desc* desc,
                        int32_t Hr, const void* W, const mf_v_desc* v, void* O,
                        void* ws, size_t ws_bytes, mf_stream_t stream);
 
+/* As mf_mapped_av, restricted to the global query blocks [qb_begin, qb_end)
+ * (global order: sequence by sequence, as row_ptr): only the O rows of those
+ * blocks are written, the rest of O is left as it was.  Uses:
+ *  - chunked prefill: a context processed in consecutive ranges gives, row for
+ *    row, the same O as one call (article, third component: the kernel works
+ *    with chunked prefill);
+ *  - prefix-partial reuse: when mf_index_lookup finds that a receiver's
+ *    context shares its first `matched` blocks with a cached sender context,
+ *    the sender's cache run over those blocks is exact for the receiver's
+ *    rows there (a causal row attends only to keys of the shared prefix);
+ *    the receiver computes its remaining rows itself.
+ *  Arguments, workspace and errors as mf_mapped_av, plus MF_ERR_INVALID_ARG
+ *  unless 0 <= qb_begin <= qb_end <= nqb_total. */
+mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc,
+                             int32_t Hr, const void* W, const mf_v_desc* v, void* O,
+                             int64_t qb_begin, int64_t qb_end, void* ws, size_t ws_bytes,
+                             mf_stream_t stream);
+
 /* Diagnostic, not on the hot path: y[i] = 2^x[i] by the FMA-pipe
  * exponential that the tensor-core block-statistics kernel uses for a share
  * of every tile's exponentials (x = j + f, j = round(x); 2^f from a degree-4

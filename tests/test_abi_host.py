@@ -187,3 +187,14 @@ def test_index_same_key_newest_wins(lib):
 def test_selftest_timeout_rejects_bad_limits(lib):
     assert lib.mf_selftest_timeout(0, None) == mfb.MF_ERR_INVALID_ARG
     assert lib.mf_selftest_timeout(5000, None) == mfb.MF_ERR_INVALID_ARG
+
+
+def test_mapped_av_range_rejects_bad_ranges(lib):
+    dsc, host = _desc()
+    P = C.c_void_p
+    cache = mfb.CsrCache(8, 36, 16, 16, 16, 16, 16, 4, 64, mfb.MF_F32, 1, 0x1000)
+    v = mfb.VDesc(16, None, 16, 0, 0, 2, 64)
+    for lo, hi in ((-1, 3), (0, 9), (5, 3)):
+        st = lib.mf_mapped_av_range(C.byref(cache), C.byref(dsc), 4, P(16), C.byref(v), P(16),
+                                    lo, hi, P(256), 1 << 20, None)
+        assert st == mfb.MF_ERR_INVALID_ARG, (lo, hi)

@@ -10,22 +10,23 @@
 //
 // One CTA owns an 8-row slice of one query block and all Hr receiver heads,
 // so every map byte is read from HBM once.  Kept key blocks are walked in
-// stages of 16 keys; a stage moves two contiguous chunks with plain bulk
-// copies: the map slab (8 rows x 16 keys x Hs heads, stored by the cache in
-// exactly the operand layout of the mixing MMA) and the V image of those 16
-// keys (prepared once per call by k_v_format).  Per stage:
+// stages of up to two 16-key groups (one where shared memory cannot hold two
+// 32-key slots); per 16-key group a stage moves two contiguous chunks with
+// plain bulk copies: the map slab (8 rows x 16 keys x Hs heads, stored by the
+// cache in exactly the operand layout of the mixing MMA) and the V image of
+// those 16 keys (prepared once per call by k_v_format).  Per 16-key group:
 //   1. mix MMA   Mix[128 pairs x Hr] = Map[128 pairs x Hs] . W^T[Hs x Hr]
 //      (tcgen05, M = 128 (row, key) pairs, K = Hs padded to a multiple of 16
-//      with zero W rows; two accumulators in TMEM);
-//   2. convert   four warps read Mix from TMEM, round to bf16 and store it as
-//      M^T_g[16 keys x 8 rows * G heads], the MN-major operand of step 3;
+//      with zero W rows; four stage accumulators in TMEM);
+//   2. convert   eight warps read Mix from TMEM, round to bf16 and store it as
+//      M^T_g[keys x 8 rows * G heads], the MN-major operand of step 3;
 //   3. O MMAs    O^T_g[128 d x 8G] += V_g^T[128 x 16] . M^T_g[16 x 8G] for every
 //      GQA group g (O^T of all groups resident in TMEM for the whole CTA).
-// A dedicated MMA warp issues every MMA with descriptors built once (only the
-// address field moves).  Converters hand each stage over through a named
-// barrier (hardware, no mbarrier round trip between warps), and mix(n + 2) is
-// issued as soon as stage n's accumulator has been read, keeping the tensor
-// core ahead of the conversion.
+// Two warps issue the MMAs, each from one elected lane, into disjoint
+// accumulators: the mix warp runs ahead (gated by the map slab and by the
+// converters releasing a mix buffer), the O warp takes each stage from the
+// converters through a named barrier.  Descriptors are built once and only
+// their address field moves.
 //
 // Why not mma.sync for the mix: on this part a legacy mma.sync takes a few
 // thousand cycles from issue to result unless hundreds are in flight; with
@@ -43,7 +44,7 @@ using namespace sm100;
 namespace av {
 
 constexpr int kRows = 8;   // query rows per CTA
-constexpr int kKeys = 16;  // keys per stage
+constexpr int kKeys = 16;  // keys per 16-key group (a stage holds one or two)
 constexpr int kD = 128;
 constexpr int kThreads = 384;  // warps 0-3 roles, 4-11 converters (two per lane quarter)
 constexpr uint32_t kTmemCols = 512;
@@ -82,7 +83,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // Named barriers 1 and 2 (by stage parity) hand stage n from the converters
-// to the MMA warp: both sides bar.sync once per stage, so neither can run a
+// to the O warp: both sides bar.sync once per stage, so neither can run a
 // phase ahead, also when a timed-out wait makes the rest of the walk a no-op.
 constexpr int kBarMt = 1;
 constexpr int kConverterWarps = 8;

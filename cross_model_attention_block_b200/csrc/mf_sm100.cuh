@@ -299,6 +299,13 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+// Three-input maximum of sm_100 (NaN inputs are ignored, as with fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Packed pair arithmetic of sm_100 (one instruction for two f32 lanes).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   float2 d;

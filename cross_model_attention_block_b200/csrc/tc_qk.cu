@@ -322,16 +322,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (MODE == kStats) {
-          // tree max and eight independent partial sums (short dependency chains)
+          // row max over the chunk with three-input maxima in eight
+          // independent chains, then eight independent partial sums
           float mx[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = v[k];
-#pragma unroll
-          for (int c = 8; c < 64; c += 8)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], v[c + k]);
-          const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sc;
+          for (int k = 0; k < 8; ++k)
+            mx[k] = fmaxf(fmax3(fmax3(fmax3(v[k], v[8 + k], v[16 + k]), v[24 + k], v[32 + k]),
+                                v[40 + k], v[48 + k]),
+                          v[56 + k]);
+          const float mt =
+              fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+              sc;
           const float m_new = valid ? fmaxf(m_run, mt) : 0.f;
           // only masked keys seen so far (m = -inf): sum nothing
           const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;

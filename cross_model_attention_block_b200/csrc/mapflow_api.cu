@@ -297,6 +297,15 @@ mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc
   return MF_OK;
 }
 
+mf_status mf_mapped_av_plan(int32_t Hs, int32_t Hr, int32_t Hkv, int32_t* out) {
+  if (!out) return fail(MF_ERR_INVALID_ARG, "out is NULL");
+  if (Hs < 8 || Hs > 64 || Hs % 8 != 0 || (Hr != 16 && Hr != 32) || Hkv < 1 || Hr % Hkv != 0 ||
+      (Hr / Hkv != 2 && Hr / Hkv != 4 && Hr / Hkv != 8))
+    return fail(MF_ERR_UNSUPPORTED, "shape outside the tensor-core fused kernel");
+  if (!mapped_av_tc_plan(Hs, Hr, Hkv, out)) return fail(MF_ERR_UNSUPPORTED, "no plan fits");
+  return MF_OK;
+}
+
 mf_status mf_exp2_fma_eval(const float* x, float* y, int64_t n, mf_stream_t stream) {
   if (n < 0 || (n > 0 && (!x || !y))) return fail(MF_ERR_INVALID_ARG, "n < 0 or NULL array");
   const cudaError_t e = launch_exp2_fma_eval(x, y, n, reinterpret_cast<cudaStream_t>(stream));

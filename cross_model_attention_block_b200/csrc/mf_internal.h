@@ -78,6 +78,9 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
                                 int64_t key_groups, int64_t qb_lo, int64_t qb_hi,
                                 cudaStream_t st);
 
+// Shared-memory plan of the tensor-core fused kernel for a shape: {KG, map
+// stages, V stages, dynamic smem bytes, offsets of map, M^T, W^T, barriers}.
+bool mapped_av_tc_plan(int Hs, int Hr, int Hkv, int32_t out[8]);
 cudaError_t launch_exp2_fma_eval(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,

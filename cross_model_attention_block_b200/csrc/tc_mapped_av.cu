@@ -516,6 +516,55 @@ __global__ void __launch_bounds__(256) k_v_format(
 
 // ------------------------------------------------------------------- host side
 
+namespace {
+// Shared-memory plan of the fused kernel for one shape: stage width (KG
+// 16-key groups), ring depths and region offsets, written into p.  Returns
+// KG, or 0 when nothing fits.  p.Hs_pad and p.G must be set.
+int plan_layout(av::Params& p, int Hs, int Hr, int Hkv, size_t& smem) {
+  p.map_bytes = 256u * uint32_t(Hs);
+  p.v_bytes = 4096u * uint32_t(Hkv);
+  p.w_bytes = (uint32_t(Hr) * uint32_t(p.Hs_pad) * 2u + 127u) & ~127u;
+  const uint32_t kb_bytes = 512u * 4u;  // kept key blocks of one row (L <= 512 B)
+  const size_t budget = 227u * 1024u - 1024u - 512u - p.w_bytes - kb_bytes;
+  // Stages of 32 keys (two 16-key groups) when two V / M^T slots and two map
+  // slots fit: half the per-stage waits, commits and hand-offs of 16-key
+  // stages.  Otherwise 16-key stages with the deepest rings that fit.
+  int kg = 0, ms = 0, vs = 0;
+  for (int cand_kg = 2; cand_kg >= 1 && ms == 0; --cand_kg) {
+    const uint32_t map_slot = (uint32_t(cand_kg) * p.map_bytes + 1024u + 1023u) & ~1023u;
+    const uint32_t mtg = uint32_t(cand_kg) * 256u * uint32_t(p.G) + 16u;
+    const uint32_t mt_bytes = (uint32_t(Hkv) * mtg + 127u) & ~127u;
+    const uint32_t v_slot = uint32_t(cand_kg) * p.v_bytes;
+    for (int cand_vs = (cand_kg == 2 ? 2 : 4); cand_vs >= 2 && ms == 0; --cand_vs) {
+      const size_t fixed = size_t(cand_vs) * (v_slot + mt_bytes);
+      for (int cand_ms = av::kMaxMapStages; cand_ms >= 2; --cand_ms)
+        if (fixed + size_t(cand_ms) * map_slot <= budget) {
+          kg = cand_kg;
+          ms = cand_ms;
+          vs = cand_vs;
+          p.map_slot = map_slot;
+          p.mt_group_stride = mtg;
+          p.mt_bytes = mt_bytes;
+          p.v_slot = v_slot;
+          break;
+        }
+    }
+  }
+  if (ms == 0) return 0;
+  p.map_stages = ms;
+  p.vm_stages = vs;
+  p.off_v = 0;
+  p.off_map = vs * p.v_slot;
+  p.off_mt = p.off_map + ms * p.map_slot;
+  p.off_w = p.off_mt + vs * p.mt_bytes;
+  p.off_kb = p.off_w + p.w_bytes;
+  p.off_bar = (p.off_kb + kb_bytes + 7u) & ~7u;
+  smem =
+      size_t(p.off_bar) + (2 * ms + 2 * vs * kg + 2 * av::kMixBufs + 1) * 8 + 32 + 1024;
+  return kg;
+}
+}  // namespace
+
 bool mapped_av_tc_supported(const mf_attn_desc& d, int Hr, const mf_v_desc& v) {
   if (d.dt != MF_BF16 || d.d != 128 || v.d != 128) return false;
   if (d.Hs % 8 != 0 || d.Hs > 64) return false;
@@ -564,46 +613,9 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
   p.G = Hr / v.Hkv;
   p.B = d.B;
   p.status = status_word();
-  p.map_bytes = 256u * uint32_t(d.Hs);
-  p.v_bytes = 4096u * uint32_t(v.Hkv);
-  p.w_bytes = (uint32_t(Hr) * uint32_t(p.Hs_pad) * 2u + 127u) & ~127u;
-  const uint32_t kb_bytes = 512u * 4u;  // kept key blocks of one row (L <= 512 B)
-  const size_t budget = 227u * 1024u - 1024u - 512u - p.w_bytes - kb_bytes;
-  // Stages of 32 keys (two 16-key groups) when two V / M^T slots and two map
-  // slots fit: half the per-stage waits, commits and hand-offs of 16-key
-  // stages.  Otherwise 16-key stages with the deepest rings that fit.
-  int kg = 0, ms = 0, vs = 0;
-  for (int cand_kg = 2; cand_kg >= 1 && ms == 0; --cand_kg) {
-    const uint32_t map_slot = (uint32_t(cand_kg) * p.map_bytes + 1024u + 1023u) & ~1023u;
-    const uint32_t mtg = uint32_t(cand_kg) * 256u * uint32_t(p.G) + 16u;
-    const uint32_t mt_bytes = (uint32_t(v.Hkv) * mtg + 127u) & ~127u;
-    const uint32_t v_slot = uint32_t(cand_kg) * p.v_bytes;
-    for (int cand_vs = (cand_kg == 2 ? 2 : 4); cand_vs >= 2 && ms == 0; --cand_vs) {
-      const size_t fixed = size_t(cand_vs) * (v_slot + mt_bytes);
-      for (int cand_ms = av::kMaxMapStages; cand_ms >= 2; --cand_ms)
-        if (fixed + size_t(cand_ms) * map_slot <= budget) {
-          kg = cand_kg;
-          ms = cand_ms;
-          vs = cand_vs;
-          p.map_slot = map_slot;
-          p.mt_group_stride = mtg;
-          p.mt_bytes = mt_bytes;
-          p.v_slot = v_slot;
-          break;
-        }
-    }
-  }
-  if (ms == 0) return cudaErrorInvalidConfiguration;
-  p.map_stages = ms;
-  p.vm_stages = vs;
-  p.off_v = 0;
-  p.off_map = vs * p.v_slot;
-  p.off_mt = p.off_map + ms * p.map_slot;
-  p.off_w = p.off_mt + vs * p.mt_bytes;
-  p.off_kb = p.off_w + p.w_bytes;
-  p.off_bar = (p.off_kb + kb_bytes + 7u) & ~7u;
-  const size_t smem =
-      size_t(p.off_bar) + (2 * ms + 2 * vs * kg + 2 * av::kMixBufs + 1) * 8 + 32 + 1024;
+  size_t smem = 0;
+  const int kg = plan_layout(p, d.Hs, Hr, v.Hkv, smem);
+  if (kg == 0) return cudaErrorInvalidConfiguration;
   const unsigned grid = unsigned(qb_hi - qb_lo) * unsigned(d.B / av::kRows);
   cudaError_t e = cudaSuccess;
 #define MF_AV(HR, G, KG)                                                                    \
@@ -625,6 +637,24 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
 #undef MF_AV_G
 #undef MF_AV
   return cudaGetLastError();
+}
+
+bool mapped_av_tc_plan(int Hs, int Hr, int Hkv, int32_t out[8]) {
+  av::Params p{};
+  p.Hs_pad = (Hs + 15) / 16 * 16;
+  p.G = Hr / Hkv;
+  size_t smem = 0;
+  const int kg = plan_layout(p, Hs, Hr, Hkv, smem);
+  if (kg == 0) return false;
+  out[0] = kg;
+  out[1] = p.map_stages;
+  out[2] = p.vm_stages;
+  out[3] = int32_t(smem);
+  out[4] = int32_t(p.off_map);
+  out[5] = int32_t(p.off_mt);
+  out[6] = int32_t(p.off_w);
+  out[7] = int32_t(p.off_bar);
+  return true;
 }
 
 }  // namespace mf

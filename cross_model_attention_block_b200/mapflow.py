@@ -28,7 +28,7 @@ EXPORTED = [
     "mf_block_stats", "mf_select_extract_workspace", "mf_select_extract",
     "mf_mapped_av_workspace", "mf_mapped_av", "mf_mapped_av_range", "mf_block_stats_noalloc",
     "mf_block_stats_noalloc_max_workspace",
-    "mf_exp2_fma_eval", "mf_selftest_timeout", "mf_sync_status", "mf_prefix_hash",
+    "mf_mapped_av_plan", "mf_exp2_fma_eval", "mf_selftest_timeout", "mf_sync_status", "mf_prefix_hash",
     "mf_index_create",
     "mf_index_destroy",
     "mf_index_insert", "mf_index_lookup", "mf_index_size",
@@ -88,6 +88,7 @@ def load_library(path: str = LIB_PATH):
         "mf_mapped_av_range": (C.c_int, [P, P, I32, P, P, P, I64, I64, P, SZ, P]),
         "mf_block_stats_noalloc_max_workspace": (SZ, []),
         "mf_block_stats_noalloc": (C.c_int, [P, P, P, P, P, P]),
+        "mf_mapped_av_plan": (C.c_int, [I32, I32, I32, P]),
         "mf_exp2_fma_eval": (C.c_int, [P, P, I64, P]),
         "mf_selftest_timeout": (C.c_int, [I32, P]),
         "mf_sync_status": (C.c_int, [P]),
@@ -286,6 +287,15 @@ def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None
                                     C.c_void_p(wsp), nbytes, _stream()))
     cache._av_ws = ws  # keep the workspace alive until the stream has used it
     return O
+
+
+def mapped_av_plan(Hs, Hr, Hkv):
+    """The fused kernel's shared-memory plan for a shape (host only): dict."""
+    out = np.zeros(8, dtype=np.int32)
+    _check(load_library().mf_mapped_av_plan(int(Hs), int(Hr), int(Hkv), out.ctypes.data))
+    keys = ("groups_per_stage", "map_stages", "v_stages", "smem_bytes", "off_map", "off_mt",
+            "off_w", "off_bar")
+    return dict(zip(keys, (int(v) for v in out)))
 
 
 def exp2_fma_eval(x):

@@ -232,6 +232,14 @@ mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc
  * NULL array with n > 0), MF_ERR_CUDA (launch failure). */
 mf_status mf_exp2_fma_eval(const float* x, float* y, int64_t n, mf_stream_t stream);
 
+/* Diagnostic, host only: the shared-memory plan the tensor-core fused kernel
+ * uses for a shape (bf16, d = 128; Hs a multiple of 8 up to 64, Hr 16 or 32,
+ * Hr / Hkv in {2, 4, 8}).  out[8] (host): 16-key groups per stage (1 or 2),
+ * map ring slots, V ring slots, dynamic shared memory in bytes, and the
+ * byte offsets of the map ring, the mixed-map ring, W^T and the barriers.
+ * Errors: MF_ERR_INVALID_ARG (NULL out), MF_ERR_UNSUPPORTED (other shapes). */
+mf_status mf_mapped_av_plan(int32_t Hs, int32_t Hr, int32_t Hkv, int32_t* out);
+
 /* Diagnostic, for tests of the failure path: launches one kernel whose
  * bounded wait (the same one every tensor-core kernel uses) waits on an
  * mbarrier phase that nothing completes, gives up after limit_ms and raises

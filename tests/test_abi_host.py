@@ -198,3 +198,34 @@ def test_mapped_av_range_rejects_bad_ranges(lib):
         st = lib.mf_mapped_av_range(C.byref(cache), C.byref(dsc), 4, P(16), C.byref(v), P(16),
                                     lo, hi, P(256), 1 << 20, None)
         assert st == mfb.MF_ERR_INVALID_ARG, (lo, hi)
+
+
+def test_fused_kernel_plan_fits_every_supported_shape(lib):
+    """The tensor-core fused kernel's shared-memory plan, for every shape it
+    accepts: within the 227 KB a CTA may use, operand rings on 1 KB
+    boundaries (128-byte-swizzled operands), at least double-buffered."""
+    seen_kg = set()
+    for Hs in range(8, 65, 8):
+        for Hr in (16, 32):
+            for G in (2, 4, 8):
+                Hkv = Hr // G
+                pl = mfb.mapped_av_plan(Hs, Hr, Hkv)
+                kg = pl["groups_per_stage"]
+                seen_kg.add(kg)
+                assert kg in (1, 2)
+                assert pl["smem_bytes"] <= 227 * 1024, (Hs, Hr, Hkv, pl)
+                assert pl["map_stages"] >= 2 and pl["v_stages"] >= 2
+                # V ring first, then map ring, mixed-map ring, W^T, barriers
+                assert pl["off_map"] == pl["v_stages"] * kg * 4096 * Hkv
+                assert pl["off_map"] % 1024 == 0
+                assert pl["off_map"] + pl["map_stages"] * kg * Hs * 256 <= pl["off_mt"]
+                assert pl["off_mt"] % 16 == 0 and pl["off_mt"] < pl["off_w"] < pl["off_bar"]
+                assert pl["off_bar"] % 8 == 0
+    assert seen_kg == {1, 2}
+    # 32-key stages where they fit, 16-key stages for big V images or big maps
+    assert mfb.mapped_av_plan(40, 32, 8)["groups_per_stage"] == 2
+    assert mfb.mapped_av_plan(40, 32, 16)["groups_per_stage"] == 1
+    assert mfb.mapped_av_plan(64, 32, 8)["groups_per_stage"] == 1
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.mapped_av_plan(40, 24, 8)
+    assert e.value.status == mfb.MF_ERR_UNSUPPORTED

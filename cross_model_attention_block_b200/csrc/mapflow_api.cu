@@ -165,6 +165,7 @@ mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
   if (e != cudaSuccess) return cuda_fail(e, "meta");
   if (sz.nqb == 0) return MF_OK;
   // the one-pass statistics keep one TMEM column per key block: 256 at most
+  // (mf_path_info reports the same choice)
   const bool tc_stats = use_tc(d) && (sz.max_len + d.B - 1) / d.B <= 256;
   e = tc_stats ? launch_stats_tc(d, sz, m, Q, K, lse, part, s)
                 : launch_stats_simt(d, sz, m, Q, K, lse, part, s);
@@ -294,6 +295,25 @@ mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc
                                            qb_begin, qb_end, s)
                      : launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, qb_begin, qb_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "mapped av");
+  return MF_OK;
+}
+
+mf_status mf_path_info(const mf_attn_desc* desc, int32_t Hr, const mf_v_desc* v,
+                       uint32_t* flags) {
+  if (!flags) return fail(MF_ERR_INVALID_ARG, "flags is NULL");
+  Sizes sz;
+  mf_status st = check_desc(desc, &sz);
+  if (st != MF_OK) return st;
+  const mf_attn_desc& d = *desc;
+  uint32_t f = 0;
+  if (use_tc(d) && (sz.max_len + d.B - 1) / d.B <= 256) f |= MF_PATH_STATS_TC;
+  if (use_tc(d)) f |= MF_PATH_EXTRACT_TC;
+  if (v) {
+    if (v->Hkv < 1 || Hr < 1 || Hr % v->Hkv != 0)
+      return fail(MF_ERR_INVALID_ARG, "Hr must be a positive multiple of Hkv");
+    if (mapped_av_tc_supported(d, Hr, *v)) f |= MF_PATH_AV_TC;
+  }
+  *flags = f;
   return MF_OK;
 }
 

@@ -28,7 +28,7 @@ EXPORTED = [
     "mf_block_stats", "mf_select_extract_workspace", "mf_select_extract",
     "mf_mapped_av_workspace", "mf_mapped_av", "mf_mapped_av_range", "mf_block_stats_noalloc",
     "mf_block_stats_noalloc_max_workspace",
-    "mf_mapped_av_plan", "mf_exp2_fma_eval", "mf_selftest_timeout", "mf_sync_status", "mf_prefix_hash",
+    "mf_mapped_av_plan", "mf_path_info", "mf_exp2_fma_eval", "mf_selftest_timeout", "mf_sync_status", "mf_prefix_hash",
     "mf_index_create",
     "mf_index_destroy",
     "mf_index_insert", "mf_index_lookup", "mf_index_size",
@@ -89,6 +89,7 @@ def load_library(path: str = LIB_PATH):
         "mf_block_stats_noalloc_max_workspace": (SZ, []),
         "mf_block_stats_noalloc": (C.c_int, [P, P, P, P, P, P]),
         "mf_mapped_av_plan": (C.c_int, [I32, I32, I32, P]),
+        "mf_path_info": (C.c_int, [P, I32, P, P]),
         "mf_exp2_fma_eval": (C.c_int, [P, P, I64, P]),
         "mf_selftest_timeout": (C.c_int, [I32, P]),
         "mf_sync_status": (C.c_int, [P]),
@@ -296,6 +297,24 @@ def mapped_av_plan(Hs, Hr, Hkv):
     keys = ("groups_per_stage", "map_stages", "v_stages", "smem_bytes", "off_map", "off_mt",
             "off_w", "off_bar")
     return dict(zip(keys, (int(v) for v in out)))
+
+
+MF_PATH_STATS_TC, MF_PATH_EXTRACT_TC, MF_PATH_AV_TC = 1, 2, 4
+
+
+def path_info(ctx: Context, Hr=None, Hkv=None):
+    """Which kernels the three calls run for a shape (host only): dict of
+    bools for the statistics, extraction and fused stages."""
+    d = ctx.desc()
+    vd = None
+    if Hr is not None:
+        vd = VDesc(0, 0, 16, 0, 0, int(Hkv), ctx.d)
+    f = C.c_uint32()
+    _check(load_library().mf_path_info(C.byref(d), int(Hr or 0),
+                                       None if vd is None else C.byref(vd), C.byref(f)))
+    return {"stats_tc": bool(f.value & MF_PATH_STATS_TC),
+            "extract_tc": bool(f.value & MF_PATH_EXTRACT_TC),
+            "mapped_av_tc": bool(f.value & MF_PATH_AV_TC)}
 
 
 def exp2_fma_eval(x):

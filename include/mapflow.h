@@ -223,14 +223,33 @@ mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc
                              mf_stream_t stream);
 
 /* Diagnostic, not on the hot path: y[i] = 2^x[i] by the FMA-pipe
- * exponential that the tensor-core block-statistics kernel uses for a share
- * of every tile's exponentials (x = j + f, j = round(x); 2^f from a degree-4
- * polynomial with relative minimax error 2.7e-6 on [-1/2, 1/2]; 2^j added to
- * the exponent).  Meant for x <= 0; x below -125 is clamped to -125.  x, y:
- * device float arrays of n elements (they may be the same array).  Lets tests
- * hold it against CUDA's exp2f.  Errors: MF_ERR_INVALID_ARG (n < 0, or a
- * NULL array with n > 0), MF_ERR_CUDA (launch failure). */
+ * exponential written for the block-statistics epilogue (x = j + f,
+ * j = round(x); 2^f from a degree-4 polynomial with relative minimax error
+ * 2.7e-6 on [-1/2, 1/2]; 2^j added to the exponent).  Measured slower there
+ * than the MUFU exponential, so the statistics kernel currently computes none
+ * of its exponentials with it.  Meant for x <= 0; x below -125 is clamped to
+ * -125.  x, y: device float arrays of n elements (they may be the same
+ * array).  Lets tests hold it against CUDA's exp2f.  Errors:
+ * MF_ERR_INVALID_ARG (n < 0, or a NULL array with n > 0), MF_ERR_CUDA (launch
+ * failure). */
 mf_status mf_exp2_fma_eval(const float* x, float* y, int64_t n, mf_stream_t stream);
+
+/* Which kernels the calls above run for a shape (host only; nothing is
+ * launched).  Every stage has a tensor-core kernel and a scalar (CUDA-core,
+ * float32 arithmetic) kernel that gives the same results more slowly:
+ *  MF_PATH_STATS_TC   mf_block_stats runs the one-pass tensor-core kernel:
+ *                     bf16, d = 128 and every sequence at most 256 key blocks
+ *                     (L_s <= 256 * B); otherwise the scalar two-pass kernel;
+ *  MF_PATH_EXTRACT_TC mf_select_extract extracts on the tensor cores: bf16,
+ *                     d = 128;
+ *  MF_PATH_AV_TC      mf_mapped_av runs the tensor-core fused kernel: bf16,
+ *                     d = 128, Hs a multiple of 8, Hr 16 or 32, Hr / Hkv in
+ *                     {2, 4, 8} (v may be NULL: this bit is then left 0).
+ * Errors: as the calls' own argument checks (MF_ERR_INVALID_ARG,
+ * MF_ERR_UNSUPPORTED), MF_ERR_INVALID_ARG for a NULL flags. */
+enum { MF_PATH_STATS_TC = 1, MF_PATH_EXTRACT_TC = 2, MF_PATH_AV_TC = 4 };
+mf_status mf_path_info(const mf_attn_desc* desc, int32_t Hr, const mf_v_desc* v,
+                       uint32_t* flags);
 
 /* Diagnostic, host only: the shared-memory plan the tensor-core fused kernel
  * uses for a shape (bf16, d = 128; Hs a multiple of 8 up to 64, Hr 16 or 32,
@@ -249,7 +268,10 @@ mf_status mf_mapped_av_plan(int32_t Hs, int32_t Hr, int32_t Hkv, int32_t* out);
 mf_status mf_selftest_timeout(int32_t limit_ms, mf_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the device status word of the
- * current device: MF_OK, MF_ERR_TIMEOUT or MF_ERR_CAPACITY. */
+ * current device: MF_OK; MF_ERR_TIMEOUT (a bounded wait gave up);
+ * MF_ERR_CAPACITY (kept blocks overflowed a CSR capacity); MF_ERR_INVALID_ARG
+ * (the fused kernel met a cache row holding more entries than its query block
+ * has key blocks, and clamped it). */
 mf_status mf_sync_status(mf_stream_t stream);
 
 /* ---- host-side prefix index (article: states are indexed by a prefix hash

@@ -2,8 +2,12 @@
 
 Tolerances (from the stated acceptance rule of the hot path):
 * kept block sets bit-exact, except query blocks whose oracle cumulative mass
-  fraction at the cut lies within 1e-4 of tau, or whose only difference is a
-  swap of blocks with oracle masses closer than 1e-6 * T; these are counted;
+  fraction at the cut lies within 1e-4 of tau ("near tau"), or whose only
+  difference swaps blocks across the cut whose oracle masses all lie within
+  1e-6 * T of the oracle's mass at the cut ("near swap"); both kinds are
+  counted, reported separately at the end of the pytest run, and the exempt
+  query block is still checked: its extracted values and its O against the
+  oracle evaluated on the GPU's own kept set;
 * O: max-abs error <= 2e-2 * max|O| for bf16, <= 1e-4 * max|O| for fp32;
 * lse, block masses and extracted probabilities: the float32 arithmetic of
   the kernels on identical (rounded) inputs; bounds are stated per check.
@@ -43,26 +47,51 @@ def kept_sets(cache):
     return rp, ci
 
 
+# Exemptions seen during this process, per label: {label: [checked, near_tau, near_swap]}.
+REPORT = {}
+
+
+def record(label, res):
+    """Add one comparison's counts to the run's exemption report."""
+    r = REPORT.setdefault(label, [0, 0, 0])
+    r[0] += res.n
+    r[1] += res.near_tau
+    r[2] += res.near_swap
+
+
 def check_selection(oracle_mass, gpu_kept, tau):
-    """0 if equal, 1 if the difference is exempt, raises otherwise."""
+    """'' if the kept sets are equal, 'near_tau' or 'near_swap' if the
+    difference is exempt; raises otherwise."""
     oracle_kept = orc.select_blocks(oracle_mass, tau)
     if list(oracle_kept) == list(gpu_kept):
-        return 0
+        return ""
     order, frac = orc.cumulative_fractions(oracle_mass)
     k = len(oracle_kept)
     near = [abs(frac[k - 1] - tau)]
     if k >= 2:
         near.append(abs(frac[k - 2] - tau))
     if min(near) < NEAR_TAU:
-        return 1
+        return "near_tau"
     T = oracle_mass.sum()
     a, b = set(oracle_kept.tolist()), set(int(x) for x in gpu_kept)
     if len(a) == len(b):
+        # swaps across the cut: oracle-kept blocks the GPU dropped, and
+        # blocks past the cut it kept, all as heavy as the cut block
+        m_cut = oracle_mass[order[k - 1]]
         diff = sorted(a ^ b)
-        if max(oracle_mass[diff]) - min(oracle_mass[diff]) < NEAR_SWAP * T:
-            return 1
+        if max(abs(oracle_mass[kb] - m_cut) for kb in diff) < NEAR_SWAP * T:
+            return "near_swap"
     raise AssertionError(f"kept sets differ beyond the exemptions: oracle {sorted(a)} "
                          f"gpu {sorted(b)}; cut fractions {near}")
+
+
+class Result(tuple):
+    """(n, exempt, worst) with the exemption kinds by name."""
+
+    def __new__(cls, n, near_tau, near_swap, worst):
+        r = super().__new__(cls, (n, near_tau + near_swap, worst))
+        r.n, r.near_tau, r.near_swap, r.worst = n, near_tau, near_swap, worst
+        return r
 
 
 def f64(t):
@@ -74,11 +103,14 @@ def block_index(cu_blk_s, qb, kb):
 
 
 def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
-                         check_values=True, lse_atol=None):
+                         check_values=True, lse_atol=None, label=None):
     """Compare the GPU result on selected (seq, qb) pairs with the oracle.
 
-    Qc, Kc, Vc, Wc are the CPU copies of the inputs (contiguous V).
-    Returns (n_checked, n_exempt, max_rel_err_O).
+    Qc, Kc, Vc, Wc are the CPU copies of the inputs (contiguous V).  The
+    extracted values and O are compared on the GPU's kept set, which equals
+    the oracle's except on counted exemptions.  Returns a Result
+    (n_checked, n_exempt, max_rel_err_O) and, with a label, adds its counts
+    to the run's exemption report.
     """
     lse_g, mass_g, cache, O_g = gpu
     B = ctx.B
@@ -92,7 +124,7 @@ def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
     mass_g = mass_g.cpu().numpy()
     W = f64(Wc)
     vals = cache.values_view() if check_values else None
-    n_ex = 0
+    n_tau = n_swap = 0
     worst = 0.0
     tol = o_tol(dtype)
     if lse_atol is None:
@@ -117,9 +149,8 @@ def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
         kept_g = ci[rp[g]:rp[g + 1]]
         assert np.all(np.diff(kept_g) > 0), "kept blocks not ascending"
         ex = check_selection(mass_o, kept_g, tau)
-        n_ex += ex
-        if ex:
-            continue
+        n_tau += ex == "near_tau"
+        n_swap += ex == "near_swap"
         # extracted probability blocks
         if check_values:
             for e, kb in zip(range(rp[g], rp[g + 1]), kept_g):
@@ -139,7 +170,10 @@ def compare_query_blocks(ctx, Qc, Kc, Vc, Wc, Hkv, tau, gpu, picks, dtype,
         err = np.abs(O_gpu - O_o).max() / scale
         worst = max(worst, err)
         assert err <= tol, f"O seq {s} qb {qb}: rel err {err:.3e} > {tol}"
-    return len(picks), n_ex, worst
+    res = Result(len(picks), n_tau, n_swap, worst)
+    if label is not None:
+        record(label, res)
+    return res
 
 
 def stored_to_logical(x, Hs, B):

@@ -6,6 +6,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from cross_model_attention_block_b200 import mapflow as mfb
 
@@ -229,3 +230,25 @@ def test_fused_kernel_plan_fits_every_supported_shape(lib):
     with pytest.raises(mfb.MapflowError) as e:
         mfb.mapped_av_plan(40, 24, 8)
     assert e.value.status == mfb.MF_ERR_UNSUPPORTED
+
+
+def test_every_bf16_workload_runs_the_tensor_core_kernels(lib):
+    """mf_path_info on the workloads' shapes: all three stages of every bf16
+    workload run on the tensor cores; the float32 one runs the scalar
+    kernels; a sequence past 256 key blocks drops the statistics to the
+    scalar two-pass kernel."""
+    from cross_model_attention_block_b200 import synth
+    for name, w in synth.workloads().items():
+        ctx = mfb.Context.make(w.lengths, w.Hs, w.d, w.B, w.band_bias, w.band_width,
+                               w.torch_dtype, device="cpu")
+        got = mfb.path_info(ctx, w.Hr, w.Hkv)
+        want = w.dtype == "bf16"
+        assert got == {"stats_tc": want, "extract_tc": want, "mapped_av_tc": want}, name
+    long = mfb.Context.make([257 * 64], 32, 128, 64, 2.0, 256, torch.bfloat16, device="cpu")
+    assert mfb.path_info(long, 32, 8) == {"stats_tc": False, "extract_tc": True,
+                                          "mapped_av_tc": True}
+    odd = mfb.Context.make([1000], 12, 128, 64, 2.0, 256, torch.bfloat16, device="cpu")
+    assert mfb.path_info(odd, 32, 8)["mapped_av_tc"] is False      # Hs not a multiple of 8
+    assert mfb.path_info(odd, 24, 8)["mapped_av_tc"] is False      # Hr not 16 or 32
+    with pytest.raises(mfb.MapflowError):
+        mfb.path_info(odd, 30, 8)                                  # Hr not a multiple of Hkv

@@ -33,6 +33,10 @@ def test_chunked_prefill_equals_one_call(args):
         mfb.mapped_av(cache, w.Hr, W, V, w.Hkv, O=O, qb_range=(a, b))
     mfb.sync_status()
     assert torch.equal(O, O_full)  # every CTA computes its rows the same way
+    # and the rows the ranges wrote are the oracle's
+    par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, (lse, mass, cache, O),
+                             par.all_picks(ctx), w.torch_dtype, check_values=False,
+                             label="chunked ranges")
 
 
 def test_range_writes_only_its_rows():
@@ -46,6 +50,9 @@ def test_range_writes_only_its_rows():
     rows[300:364] = True
     assert torch.equal(O[rows], O_full[rows])
     assert bool((O[~rows] == 7.0).all())
+    par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, (lse, mass, cache, O),
+                             [(0, 2), (0, 3), (0, 4), (1, 0)], w.torch_dtype,
+                             check_values=False, label="chunked ranges")
     with pytest.raises(mfb.MapflowError):
         mfb.mapped_av(cache, w.Hr, x.W.cuda(), x.V.cuda(), w.Hkv, O=O, qb_range=(3, 99))
 
@@ -75,3 +82,9 @@ def test_prefix_partial_reuse_through_the_index():
     n = matched * B
     assert torch.equal(O[:n], O_ref[:n])
     assert bool((O[n:] == 7.0).all())
+    # the oracle on the receiver's side: the sender's map over the shared
+    # prefix (the receiver's rows there attend only to prefix keys) times the
+    # receiver's own V
+    par.compare_query_blocks(ctx, x.Q, x.K, Vr.cpu(), x.W, w.Hkv, w.tau,
+                             (lse, mass, cache, O), [(0, qb) for qb in range(matched)],
+                             w.torch_dtype, check_values=False, label="prefix reuse")

@@ -282,3 +282,85 @@ def test_extracted_blocks_are_the_probabilities():
             if kb == qb:  # upper triangle of the diagonal block is zero
                 for i in range(blk.shape[1]):
                     assert np.all(blk[:, i, i + 1:] == 0.0)
+
+
+# ------------------------------------------- cumulative fractions (exemptions)
+
+def _check_cumulative_fractions(fn, mass, tau):
+    """What the selection rule fixes about (order, c_k / T), independent of the
+    oracle: the order is numpy's lexicographic sort by (-mass, index); the
+    fractions are the running sums in that order over the plain total; and the
+    cut of select_blocks sits where the fraction first reaches tau."""
+    order, frac = fn(mass)
+    n = len(mass)
+    ref_order = np.lexsort((np.arange(n), -mass))          # last key is primary
+    assert list(order) == list(ref_order), "order is not (mass desc, index asc)"
+    total = math.fsum(mass)
+    run = 0.0
+    for k, kb in enumerate(ref_order):
+        run += mass[kb]
+        assert abs(frac[k] - run / total) <= 1e-12, f"fraction {k} is not c_k / T"
+    assert abs(frac[-1] - 1.0) <= 1e-12
+    kept = orc.select_blocks(mass, tau)
+    k = len(kept)
+    assert set(kept.tolist()) == set(order[:k].tolist())
+    if tau < 1.0:
+        assert frac[k - 1] >= tau - 1e-12
+        assert k == 1 or frac[k - 2] < tau
+
+
+def _mass_cases():
+    rng = np.random.default_rng(300)
+    cases = []
+    for _ in range(8):
+        n = int(rng.integers(2, 40))
+        cases.append((rng.exponential(size=n) ** 2, float(rng.uniform(0.3, 0.99))))
+    # exact ties: Q = 0 block masses (blocks fully in the past tie)
+    Q = np.zeros((64, 1, 4))
+    K = np.random.default_rng(11).standard_normal((64, 1, 4))
+    _, _, mass = orc.query_block(Q, K, 7, 8, 0.0, 256)
+    cases.append((mass, 0.5))
+    cases.append((np.array([3.0, 1.0, 3.0, 2.0, 1.0]), 0.6))
+    return cases
+
+
+def test_cumulative_fractions_order_and_cut():
+    for mass, tau in _mass_cases():
+        _check_cumulative_fractions(orc.cumulative_fractions, mass, tau)
+
+
+def _mutant_ascending(mass):
+    order = sorted(range(len(mass)), key=lambda kb: (mass[kb], kb))
+    c = np.cumsum(np.array([mass[kb] for kb in order]))
+    return np.array(order), c / c[-1]
+
+
+def _mutant_ties_high(mass):
+    order = sorted(range(len(mass)), key=lambda kb: (-mass[kb], -kb))
+    c = np.cumsum(np.array([mass[kb] for kb in order]))
+    return np.array(order), c / c[-1]
+
+
+def _mutant_shifted(mass):
+    order, frac = orc.cumulative_fractions(mass)
+    return order, np.concatenate([[0.0], frac[:-1]])       # c_{k-1} in place of c_k
+
+
+def _mutant_wrong_total(mass):
+    order, frac = orc.cumulative_fractions(mass)
+    return order, frac * (1.0 - 1.0 / len(mass))           # divided by a larger total
+
+
+@pytest.mark.parametrize("mutant", [_mutant_ascending, _mutant_ties_high, _mutant_shifted,
+                                    _mutant_wrong_total])
+def test_cumulative_fraction_pins_catch_planted_mistakes(mutant):
+    """Each plausible mistake planted in a copy of the oracle function fails
+    the checks above on at least one of the cases."""
+    failed = False
+    for mass, tau in _mass_cases():
+        try:
+            _check_cumulative_fractions(mutant, mass, tau)
+        except AssertionError:
+            failed = True
+            break
+    assert failed

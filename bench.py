@@ -9,8 +9,11 @@ larger than L2, so no separate L2 flush is done.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (torchrun), every rank runs an independent replica of the layer
-(the path has no exchange step): weak scaling, time = max over ranks.
+With N > 1 (torchrun), the layer's query blocks are split across the ranks
+with no data-path collective (every query block's work is independent): a
+single sequence in zig-zag pairs (qb, nqb-1-qb), a varlen batch by whole
+sequences balanced by causal cost.  The total work is fixed as N grows
+(strong scaling); time = max over ranks.
 `--impl reference` times the CPU oracle on the host cores on a bounded
 sample of the same workload (rank 0 only).
 """
@@ -30,6 +33,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from cross_model_attention_block_b200 import partition  # noqa: E402
 from cross_model_attention_block_b200 import synth  # noqa: E402
 
 METRIC = ("mapped-AV GB/s & % HBM roofline; compress tokens/s & % tensor peak; "
@@ -168,7 +172,7 @@ def bench_reference(args, wl):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "tokens": L, "Hs": wl.Hs, "Hr": wl.Hr,
                    "Hkv": wl.Hkv, "d": wl.d, "B": wl.B, "tau": wl.tau},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -211,20 +215,58 @@ def cpu_baseline_sample(wl, x, budget_s=20.0):
 
 # ----------------------------------------------------------------- our arm
 
-def algorithmic(wl, nnz):
-    """Per-launch algorithmic bytes / flops of the three kernels."""
-    L = wl.ntok
-    pairs = sum(l * (l + 1) // 2 for l in wl.lengths)
+def rank_plan(wl, rank, world):
+    """Global query-block ranges [(begin, end), ...] this rank runs: the whole
+    context at N = 1; zig-zag pairs of one sequence, or whole sequences of a
+    varlen batch balanced by causal cost, at N > 1."""
+    nq = [(L + wl.B - 1) // wl.B for L in wl.lengths]
+    if world == 1:
+        return [(0, sum(nq))]
+    if len(wl.lengths) == 1:
+        return partition.zigzag_ranges(nq[0], world, rank)
+    cu = np.concatenate([[0], np.cumsum(nq)])
+    out = []
+    for s in partition.balance_sequences(wl.lengths, world, rank):
+        a, b = int(cu[s]), int(cu[s + 1])
+        if a == b:
+            continue
+        if out and out[-1][1] == a:
+            out[-1] = (out[-1][0], b)
+        else:
+            out.append((a, b))
+    return out
+
+
+def plan_units(wl, ranges):
+    """(rows, causal (i, j) pairs) of the query blocks in `ranges`."""
+    nq = [(L + wl.B - 1) // wl.B for L in wl.lengths]
+    cu = np.concatenate([[0], np.cumsum(nq)])
+    rows = pairs = 0
+    for a, b in ranges:
+        for g in range(a, b):
+            s = int(np.searchsorted(cu, g, side="right") - 1)
+            L, qb = wl.lengths[s], g - int(cu[s])
+            i0, i1 = qb * wl.B, min(L, (qb + 1) * wl.B)
+            rows += i1 - i0
+            pairs += (i1 * (i1 + 1) - i0 * (i0 + 1)) // 2
+    return rows, pairs
+
+
+def algorithmic(wl, nnz, ranges=None):
+    """Algorithmic bytes / flops of the three kernels over the query blocks of
+    `ranges` (the whole context by default): one launch each at N = 1."""
+    rows, pairs = plan_units(wl, ranges or [(0, sum((L + wl.B - 1) // wl.B
+                                                    for L in wl.lengths))])
     el = 2 if wl.dtype == "bf16" else 4
     nqb = sum((l + wl.B - 1) // wl.B for l in wl.lengths)
     map_bytes = nnz * wl.Hs * wl.B * wl.B * el
-    av_bytes = (map_bytes + L * wl.Hkv * wl.d * el + L * wl.Hr * wl.d * el
+    av_bytes = (map_bytes + wl.ntok * wl.Hkv * wl.d * el + rows * wl.Hr * wl.d * el
                 + wl.Hr * wl.Hs * el + 4 * nnz + 8 * (nqb + 1))
     stats_flops = 2.0 * wl.d * pairs * wl.Hs          # one QK^T over the causal triangle
     extract_bytes = map_bytes
     av_flops = 2.0 * nnz * wl.B * wl.B * (wl.Hs * wl.Hr + wl.d * wl.Hr)
     return dict(av_bytes=av_bytes, stats_flops=stats_flops, extract_bytes=extract_bytes,
-                av_flops=av_flops, map_bytes=map_bytes)
+                av_flops=av_flops, map_bytes=map_bytes, rows=rows)
 
 
 def dense_attention_ms(wl, dev, stream, ev, warmup, steps):
@@ -282,31 +324,42 @@ def bench_ours(args, wl, rank, world, local_rank):
                            wl.torch_dtype, device=dev)
     Q, K, V, W = (t.to(dev) for t in (x.Q, x.K, x.V, x.W))
     nqb, nblocks = ctx.layout_sizes()
+    plan = rank_plan(wl, rank, world)
     lse = torch.empty((wl.Hs, wl.ntok), dtype=torch.float32, device=dev)
     mass = torch.empty((nblocks,), dtype=torch.float32, device=dev)
-    cache = mfb.Cache(ctx, device=dev)
+    # one cache per range, sized to the range's causal blocks
+    caches = [mfb.Cache(ctx, capacity=ctx.range_blocks(a, b), device=dev) for a, b in plan]
     O = torch.empty((wl.ntok, wl.Hr, wl.d), dtype=wl.torch_dtype, device=dev)
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
-    def step(marks=None):
+    def run(Qd, Kd, Vd, Wd, marks=None):
+        # stage by stage over this rank's ranges: statistics, then selection
+        # and extraction, then the fused kernel
         if marks is not None:
             marks[0].record(stream)
-        mfb.block_stats(ctx, Q, K, lse=lse, mass=mass)
+        for r in plan:
+            mfb.block_stats(ctx, Qd, Kd, lse=lse, mass=mass, qb_range=r)
         if marks is not None:
             marks[1].record(stream)
-        mfb.select_extract(ctx, Q, K, lse, mass, wl.tau, cache=cache)
+        for r, c in zip(plan, caches):
+            mfb.select_extract(ctx, Qd, Kd, lse, mass, wl.tau, cache=c, qb_range=r)
         if marks is not None:
             marks[2].record(stream)
-        mfb.mapped_av(cache, wl.Hr, W, V, wl.Hkv, O=O, workspace=getattr(cache, "_av_ws", None))
+        for r, c in zip(plan, caches):
+            mfb.mapped_av(c, wl.Hr, Wd, Vd, wl.Hkv, O=O, workspace=getattr(c, "_av_ws", None),
+                          qb_range=r)
         if marks is not None:
             marks[3].record(stream)
+
+    def step(marks=None):
+        run(Q, K, V, W, marks)
 
     for _ in range(args.warmup):
         step()
     mfb.sync_status()
-    nnz = cache.nnz
-    alg = algorithmic(wl, nnz)
+    nnz = sum(c.nnz for c in caches)
+    alg = algorithmic(wl, nnz, plan)
 
     marks = [[ev() for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
@@ -346,10 +399,7 @@ def bench_ours(args, wl, rank, world, local_rank):
         dK.copy_(hK, non_blocking=True)
         dV.copy_(hV, non_blocking=True)
         dW.copy_(hW, non_blocking=True)
-        mfb.block_stats(ctx, dQ, dK, lse=lse, mass=mass)
-        mfb.select_extract(ctx, dQ, dK, lse, mass, wl.tau, cache=cache)
-        mfb.mapped_av(cache, wl.Hr, dW, dV, wl.Hkv, O=O,
-                      workspace=getattr(cache, "_av_ws", None))
+        run(dQ, dK, dV, dW)
         hO.copy_(O, non_blocking=True)
 
     e2e_step()
@@ -369,7 +419,7 @@ def bench_ours(args, wl, rank, world, local_rank):
         return
     peaks, src = load_peaks()
     ms_step = ms / args.steps
-    tokens = wl.ntok * world
+    tokens = wl.ntok  # one layer, split across the ranks
     t_stats, t_sel, t_av = stage_ms
     av_gbs = alg["av_bytes"] / (t_av * 1e-3) / 1e9
     stats_tf = alg["stats_flops"] / (t_stats * 1e-3) / 1e12
@@ -402,14 +452,15 @@ def bench_ours(args, wl, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": tokens / (ms_step * 1e-3), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "tokens": wl.ntok, "Hs": wl.Hs, "Hr": wl.Hr,
                    "Hkv": wl.Hkv, "d": wl.d, "B": wl.B, "tau": wl.tau,
                    "kept_blocks": nnz, "causal_blocks": nblocks,
                    "map_gb": alg["map_bytes"] / 1e9,
                    "l2": "inputs larger than L2 (kept map >> 126 MB); no flush",
-                   "parallelism": f"replicas{world}"},
+                   "parallelism": (f"query-block ranges x{world} (rank 0: {plan})"
+                                   if world > 1 else "single GPU")},
         "mapped_av_gbs": av_gbs, "mapped_av_hbm_frac": av_gbs / hbm,
         "compress_tokens_per_s": wl.ntok / ((t_stats + t_sel) * 1e-3),
         "stats_tensor_frac": stats_tf / tens,
@@ -421,17 +472,17 @@ def bench_ours(args, wl, rank, world, local_rank):
         "clocks": clk,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * LAUNCHES_PER_STEP,
+        "gpu_launches": args.steps * LAUNCHES_PER_RANGE * len(plan),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_sample(wl, x)
     print(json.dumps(line), flush=True)
 
 
-# kernels of ours launched per step: stats (meta, stats, mass reduce), select and
-# extract (meta, qb map, select, scan, fill, extract), mapped AV (group meta,
-# V regrouping, fused kernel)
-LAUNCHES_PER_STEP = 12
+# kernels of ours launched per query-block range and step: stats (meta, stats,
+# mass reduce), select and extract (meta, qb map, select, scan, fill,
+# extract), mapped AV (group meta, V regrouping, fused kernel)
+LAUNCHES_PER_RANGE = 12
 
 
 def main(argv=None):

@@ -2,6 +2,7 @@
 // kernels, the device status word and the host prefix-hash index.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -91,6 +92,41 @@ static size_t meta_bytes(Carve& c, int nseq, int64_t ntiles, Meta* m) {
   return c.used;
 }
 
+// Tiles and block span of the global query blocks [lo, hi) (host arithmetic
+// on cu_seqlens_host; the same tile rule as k_meta).
+static QbRange range_of(const mf_attn_desc& d, const Sizes& sz, int64_t lo, int64_t hi) {
+  QbRange r;
+  r.qb_lo = lo;
+  r.qb_hi = hi;
+  r.blk_lo = r.blk_hi = sz.nblocks;
+  const int per = 128 / d.B;
+  int64_t q0 = 0, b0 = 0;
+  bool first = true;
+  for (int s = 0; s < d.nseq; ++s) {
+    const int64_t L = int64_t(d.cu_seqlens_host[s + 1]) - d.cu_seqlens_host[s];
+    const int64_t n = (L + d.B - 1) / d.B;
+    const int64_t a = std::max(lo - q0, int64_t(0)), e = std::min(hi - q0, n);
+    if (a < e) {
+      r.ntiles += (e - 1) / per - a / per + 1;
+      if (first) {
+        r.blk_lo = b0 + a * (a + 1) / 2;
+        first = false;
+      }
+      r.blk_hi = b0 + e * (e + 1) / 2;
+    }
+    q0 += n;
+    b0 += n * (n + 1) / 2;
+  }
+  if (first) r.blk_lo = r.blk_hi = 0;
+  return r;
+}
+
+static mf_status check_range(const Sizes& sz, int64_t lo, int64_t hi) {
+  if (lo < 0 || lo > hi || hi > sz.nqb)
+    return fail(MF_ERR_INVALID_ARG, "query-block range outside [0, nqb_total]");
+  return MF_OK;
+}
+
 // bf16 with d = 128 runs on the tcgen05 kernels; float32 (1e-4 relative
 // accuracy) and d = 64 run on the scalar kernels.
 static bool use_tc(const mf_attn_desc& d) { return d.dt == MF_BF16 && d.d == 128; }
@@ -152,7 +188,18 @@ mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
   Sizes sz;
   mf_status st = check_desc(desc, &sz);
   if (st != MF_OK) return st;
+  return mf_block_stats_range(desc, Q, K, lse, mass, 0, sz.nqb, ws, ws_bytes, stream);
+}
+
+mf_status mf_block_stats_range(const mf_attn_desc* desc, const void* Q, const void* K,
+                               float* lse, float* mass, int64_t qb_begin, int64_t qb_end,
+                               void* ws, size_t ws_bytes, mf_stream_t stream) {
+  Sizes sz;
+  mf_status st = check_desc(desc, &sz);
+  if (st != MF_OK) return st;
   if (!Q || !K || !lse || !mass) return fail(MF_ERR_INVALID_ARG, "Q, K, lse or mass is NULL");
+  st = check_range(sz, qb_begin, qb_end);
+  if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
   if (!ws || !aligned256(ws) || ws_bytes < stats_ws(d, sz, nullptr, nullptr, nullptr))
     return fail(MF_ERR_WORKSPACE, "workspace missing, not 256-byte aligned or too small");
@@ -161,16 +208,17 @@ mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
   Meta m;
   float* part = nullptr;
   stats_ws(d, sz, ws, &m, &part);
-  cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, m, s);
+  const QbRange r = range_of(d, sz, qb_begin, qb_end);
+  cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, r.qb_lo, r.qb_hi, m, s);
   if (e != cudaSuccess) return cuda_fail(e, "meta");
-  if (sz.nqb == 0) return MF_OK;
+  if (r.qb_hi == r.qb_lo) return MF_OK;
   // the one-pass statistics keep one TMEM column per key block: 256 at most
   // (mf_path_info reports the same choice)
   const bool tc_stats = use_tc(d) && (sz.max_len + d.B - 1) / d.B <= 256;
-  e = tc_stats ? launch_stats_tc(d, sz, m, Q, K, lse, part, s)
-                : launch_stats_simt(d, sz, m, Q, K, lse, part, s);
+  e = tc_stats ? launch_stats_tc(d, sz, r, m, Q, K, lse, part, s)
+                : launch_stats_simt(d, sz, r, m, Q, K, lse, part, s);
   if (e != cudaSuccess) return cuda_fail(e, "block stats");
-  e = launch_mass_reduce(part, d.Hs, sz.nblocks, mass, s);
+  e = launch_mass_reduce(part, d.Hs, sz.nblocks, r.blk_lo, r.blk_hi, mass, s);
   if (e != cudaSuccess) return cuda_fail(e, "mass reduce");
   return MF_OK;
 }
@@ -199,10 +247,23 @@ mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void*
   Sizes sz;
   mf_status st = check_desc(desc, &sz);
   if (st != MF_OK) return st;
+  return mf_select_extract_range(desc, Q, K, lse, mass, tau, out, 0, sz.nqb, ws, ws_bytes,
+                                 stream);
+}
+
+mf_status mf_select_extract_range(const mf_attn_desc* desc, const void* Q, const void* K,
+                                  const float* lse, const float* mass, double tau,
+                                  mf_csr_cache* out, int64_t qb_begin, int64_t qb_end, void* ws,
+                                  size_t ws_bytes, mf_stream_t stream) {
+  Sizes sz;
+  mf_status st = check_desc(desc, &sz);
+  if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
   if (!Q || !K || !lse || !mass) return fail(MF_ERR_INVALID_ARG, "Q, K, lse or mass is NULL");
   if (!(tau > 0.0) || !std::isfinite(tau)) return fail(MF_ERR_INVALID_ARG, "tau must be > 0");
   st = check_cache(out, d, sz);
+  if (st != MF_OK) return st;
+  st = check_range(sz, qb_begin, qb_end);
   if (st != MF_OK) return st;
   if (!ws || !aligned256(ws) ||
       ws_bytes < select_ws(d, sz, nullptr, nullptr, nullptr, nullptr, nullptr))
@@ -214,17 +275,18 @@ mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void*
   uint8_t* keep = nullptr;
   int32_t* slot = nullptr;
   select_ws(d, sz, ws, &m, &counts, &keep, &slot);
-  cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, m, s);
+  const QbRange r = range_of(d, sz, qb_begin, qb_end);
+  cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, r.qb_lo, r.qb_hi, m, s);
   if (e != cudaSuccess) return cuda_fail(e, "meta");
   if (sz.nqb == 0) {
     e = cudaMemsetAsync(out->row_ptr, 0, sizeof(int64_t), s);
     return e == cudaSuccess ? MF_OK : cuda_fail(e, "row_ptr");
   }
-  e = launch_select(d, sz, m, mass, tau, *out, counts, keep, slot, s);
+  e = launch_select(d, sz, r, m, mass, tau, *out, counts, keep, slot, s);
   if (e != cudaSuccess) return cuda_fail(e, "select");
-  e = use_tc(d) ? launch_extract_tc(d, sz, m, Q, K, lse, slot, out->values,
+  e = use_tc(d) ? launch_extract_tc(d, sz, r, m, Q, K, lse, slot, out->values,
                                     out->nnz_capacity, s)
-                : launch_extract_simt(d, sz, Q, K, lse, *out, s);
+                : launch_extract_simt(d, sz, r, Q, K, lse, *out, s);
   if (e != cudaSuccess) return cuda_fail(e, "extract");
   return MF_OK;
 }
@@ -282,8 +344,8 @@ mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc
   if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
   if (!W || !O) return fail(MF_ERR_INVALID_ARG, "W or O is NULL");
-  if (qb_begin < 0 || qb_begin > qb_end || qb_end > sz.nqb)
-    return fail(MF_ERR_INVALID_ARG, "query-block range outside [0, nqb_total]");
+  st = check_range(sz, qb_begin, qb_end);
+  if (st != MF_OK) return st;
   const bool tc = mapped_av_tc_supported(d, Hr, *v);
   if (tc && (!ws || !aligned256(ws) ||
              ws_bytes < mapped_av_tc_workspace(d.nseq, key_groups(d), v->Hkv)))

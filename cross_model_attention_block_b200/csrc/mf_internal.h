@@ -36,6 +36,15 @@ struct Sizes {
   int32_t max_len = 0;
 };
 
+// A range of global query blocks [qb_lo, qb_hi) of a context: the 128-row
+// tiles that hold at least one of its query blocks, and the range of block
+// indices [blk_lo, blk_hi) of its blocks (contiguous in the mass layout).
+struct QbRange {
+  int64_t qb_lo = 0, qb_hi = 0;
+  int64_t blk_lo = 0, blk_hi = 0;
+  int64_t ntiles = 0;
+};
+
 // Bump allocator over a caller workspace (256-byte aligned pieces).
 struct Carve {
   char* base;
@@ -51,15 +60,17 @@ struct Carve {
 };
 
 // ---- launchers (return cudaGetLastError of the launch) ----
-cudaError_t launch_meta(int nseq, const int32_t* cu_seqlens, int B, const Meta& m,
-                        cudaStream_t st);
+// The tile list holds the tiles of the query blocks [qb_lo, qb_hi) only.
+cudaError_t launch_meta(int nseq, const int32_t* cu_seqlens, int B, int64_t qb_lo,
+                        int64_t qb_hi, const Meta& m, cudaStream_t st);
 
-// Tensor-core kernels (bf16, d = 128).
-cudaError_t launch_stats_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                            const void* Q, const void* K, float* lse, float* part,
-                            cudaStream_t st);
-cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                              const void* Q, const void* K, const float* lse,
+// Tensor-core kernels (bf16, d = 128), over the query blocks of a range: they
+// write lse rows, partial masses and cache entries of those blocks only.
+cudaError_t launch_stats_tc(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                            const Meta& m, const void* Q, const void* K, float* lse,
+                            float* part, cudaStream_t st);
+cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                              const Meta& m, const void* Q, const void* K, const float* lse,
                               const int32_t* slot, void* values, int64_t capacity,
                               cudaStream_t st);
 
@@ -83,19 +94,22 @@ cudaError_t launch_mapped_av_tc(const mf_csr_cache& c, const mf_attn_desc& d, co
 bool mapped_av_tc_plan(int Hs, int Hr, int Hkv, int32_t out[8]);
 cudaError_t launch_exp2_fma_eval(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint64_t limit_ns, cudaStream_t st);
-cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                              const void* Q, const void* K, float* lse, float* part,
-                              cudaStream_t st);
-cudaError_t launch_mass_reduce(const float* part, int Hs, int64_t nblocks, float* mass,
-                               cudaStream_t st);
+cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                              const Meta& m, const void* Q, const void* K, float* lse,
+                              float* part, cudaStream_t st);
+// mass[b] = sum_h part[h][b] for the blocks b in [blk_lo, blk_hi).
+cudaError_t launch_mass_reduce(const float* part, int Hs, int64_t nblocks, int64_t blk_lo,
+                               int64_t blk_hi, float* mass, cudaStream_t st);
 
-cudaError_t launch_select(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                          const float* mass, double tau, const mf_csr_cache& c,
+// Selection of the query blocks of a range; the CSR rows of every other query
+// block are left empty.
+cudaError_t launch_select(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                          const Meta& m, const float* mass, double tau, const mf_csr_cache& c,
                           int32_t* counts, uint8_t* keep, int32_t* slot, cudaStream_t st);
 
-cudaError_t launch_extract_simt(const mf_attn_desc& d, const Sizes& sz, const void* Q,
-                                const void* K, const float* lse, const mf_csr_cache& c,
-                                cudaStream_t st);
+cudaError_t launch_extract_simt(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                                const void* Q, const void* K, const float* lse,
+                                const mf_csr_cache& c, cudaStream_t st);
 
 cudaError_t launch_mapped_av_simt(const mf_csr_cache& c, const mf_attn_desc& d,
                                   const Sizes& sz, int Hr, const void* W,

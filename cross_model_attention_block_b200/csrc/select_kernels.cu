@@ -34,11 +34,12 @@ __device__ __forceinline__ bool precedes(float ma, int ia, float mb, int ib) {
 __global__ void __launch_bounds__(kSelThreads) k_select(
     const float* __restrict__ mass, const int64_t* __restrict__ cu_blk,
     const int32_t* __restrict__ qb_seq, const int32_t* __restrict__ qb_idx, double tau,
-    int32_t* __restrict__ counts, uint8_t* __restrict__ keep) {
+    int64_t qb_lo, int32_t* __restrict__ counts, uint8_t* __restrict__ keep) {
   __shared__ float mv[kSelMax];
   __shared__ int kv[kSelMax];
   __shared__ int kstar_s;
-  const int gqb = blockIdx.x, tid = threadIdx.x;
+  const int64_t gqb = qb_lo + blockIdx.x;
+  const int tid = threadIdx.x;
   const int s = qb_seq[gqb], qb = qb_idx[gqb];
   const int n = qb + 1;
   const int64_t blk0 = cu_blk[s] + int64_t(qb) * (qb + 1) / 2;
@@ -113,10 +114,10 @@ __global__ void __launch_bounds__(1024) k_scan(const int32_t* __restrict__ count
 // Ascending column indices and the block -> entry map (-1 when not kept).
 __global__ void k_fill(const int64_t* __restrict__ row_ptr, const uint8_t* __restrict__ keep,
                        const int64_t* __restrict__ cu_blk, const int32_t* __restrict__ qb_seq,
-                       const int32_t* __restrict__ qb_idx, int64_t capacity,
+                       const int32_t* __restrict__ qb_idx, int64_t capacity, int64_t qb_lo,
                        int32_t* __restrict__ col_idx, int32_t* __restrict__ slot,
                        unsigned* status) {
-  const int gqb = blockIdx.x;
+  const int64_t gqb = qb_lo + blockIdx.x;
   if (threadIdx.x != 0) return;
   const int s = qb_seq[gqb], qb = qb_idx[gqb];
   const int64_t blk0 = cu_blk[s] + int64_t(qb) * (qb + 1) / 2;
@@ -138,17 +139,24 @@ __global__ void k_fill(const int64_t* __restrict__ row_ptr, const uint8_t* __res
   if (over) atomicOr(status, kStatusCapacity);
 }
 
-cudaError_t launch_select(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                          const float* mass, double tau, const mf_csr_cache& c,
+cudaError_t launch_select(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                          const Meta& m, const float* mass, double tau, const mf_csr_cache& c,
                           int32_t* counts, uint8_t* keep, int32_t* slot, cudaStream_t st) {
   if (sz.nqb == 0) return cudaSuccess;
   int g = int(std::min<int64_t>((sz.nqb + 255) / 256, 1024));
   k_qb_map<<<g, 256, 0, st>>>(sz.nqb, d.nseq, m.cu_qb, c.qb_seq, c.qb_idx);
-  k_select<<<unsigned(sz.nqb), kSelThreads, 0, st>>>(mass, m.cu_blk, c.qb_seq, c.qb_idx, tau,
-                                                     counts, keep);
+  const unsigned n = unsigned(r.qb_hi - r.qb_lo);
+  if (n < sz.nqb) {  // rows outside the range stay empty
+    cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * size_t(sz.nqb), st);
+    if (e != cudaSuccess) return e;
+  }
+  if (n > 0)
+    k_select<<<n, kSelThreads, 0, st>>>(mass, m.cu_blk, c.qb_seq, c.qb_idx, tau, r.qb_lo,
+                                        counts, keep);
   k_scan<<<1, 1024, 0, st>>>(counts, sz.nqb, c.row_ptr);
-  k_fill<<<unsigned(sz.nqb), 32, 0, st>>>(c.row_ptr, keep, m.cu_blk, c.qb_seq, c.qb_idx,
-                                          c.nnz_capacity, c.col_idx, slot, status_word());
+  if (n > 0)
+    k_fill<<<n, 32, 0, st>>>(c.row_ptr, keep, m.cu_blk, c.qb_seq, c.qb_idx, c.nnz_capacity,
+                             r.qb_lo, c.col_idx, slot, status_word());
   return cudaGetLastError();
 }
 

@@ -20,8 +20,9 @@ namespace mf {
 
 // ---------------------------------------------------------------- metadata
 
-__global__ void k_meta(int nseq, const int32_t* __restrict__ cu_seqlens, int B, int32_t* cu_qb,
-                       int64_t* cu_blk, int32_t* cu_tile, int32_t* tiles) {
+__global__ void k_meta(int nseq, const int32_t* __restrict__ cu_seqlens, int B, int64_t qb_lo,
+                       int64_t qb_hi, int32_t* cu_qb, int64_t* cu_blk, int32_t* cu_tile,
+                       int32_t* tiles) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   int32_t q = 0, t = 0, tmax = 0;
   int64_t b = 0;
@@ -40,20 +41,26 @@ __global__ void k_meta(int nseq, const int32_t* __restrict__ cu_seqlens, int B, 
     cu_blk[s + 1] = b;
     cu_tile[s + 1] = t;
   }
-  // 128-row tiles ordered by tile index descending (longest causal rows first)
+  // 128-row tiles ordered by tile index descending (longest causal rows
+  // first), only those holding a query block of [qb_lo, qb_hi)
+  const int per = 128 / B;  // query blocks per tile
   int w = 0;
   for (int tt = tmax - 1; tt >= 0; --tt)
     for (int s = 0; s < nseq; ++s)
       if (tt < cu_tile[s + 1] - cu_tile[s]) {
+        const int64_t a = cu_qb[s] + int64_t(tt) * per;                 // first query block
+        const int64_t e = min(int64_t(cu_qb[s + 1]), a + per);           // past the last
+        if (a >= qb_hi || e <= qb_lo) continue;
         tiles[2 * w] = s;
         tiles[2 * w + 1] = tt;
         ++w;
       }
 }
 
-cudaError_t launch_meta(int nseq, const int32_t* cu_seqlens, int B, const Meta& m,
-                        cudaStream_t st) {
-  k_meta<<<1, 32, 0, st>>>(nseq, cu_seqlens, B, m.cu_qb, m.cu_blk, m.cu_tile, m.tiles);
+cudaError_t launch_meta(int nseq, const int32_t* cu_seqlens, int B, int64_t qb_lo,
+                        int64_t qb_hi, const Meta& m, cudaStream_t st) {
+  k_meta<<<1, 32, 0, st>>>(nseq, cu_seqlens, B, qb_lo, qb_hi, m.cu_qb, m.cu_blk, m.cu_tile,
+                           m.tiles);
   return cudaGetLastError();
 }
 
@@ -77,12 +84,13 @@ __global__ void __launch_bounds__(128) k_stats_simt(
     const T* __restrict__ Q, const T* __restrict__ K, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ cu_qb, const int64_t* __restrict__ cu_blk, int nseq, int Hs,
     int B, float scale, float band_bias, int band_width, int64_t ntok, int64_t nblocks,
-    float* __restrict__ lse_out, float* __restrict__ part) {
+    int64_t qb_lo, float* __restrict__ lse_out, float* __restrict__ part) {
   __shared__ float ks[kKeyTile][D + 1];
   __shared__ float red[4];
-  const int gqb = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int64_t gqb = qb_lo + blockIdx.x;
+  const int h = blockIdx.y, tid = threadIdx.x;
   const int s = upper_index(cu_qb, nseq, gqb);
-  const int qb = gqb - cu_qb[s];
+  const int qb = int(gqb - cu_qb[s]);
   const int seq0 = cu_seqlens[s];
   const int L = cu_seqlens[s + 1] - seq0;
   const int i = qb * B + tid;
@@ -157,15 +165,17 @@ __global__ void __launch_bounds__(128) k_stats_simt(
   }
 }
 
-cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                              const void* Q, const void* K, float* lse, float* part,
-                              cudaStream_t st) {
-  dim3 grid(unsigned(sz.nqb), unsigned(d.Hs));
+cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                              const Meta& m, const void* Q, const void* K, float* lse,
+                              float* part, cudaStream_t st) {
+  if (r.qb_hi <= r.qb_lo) return cudaSuccess;
+  dim3 grid(unsigned(r.qb_hi - r.qb_lo), unsigned(d.Hs));
   const float scale = 1.0f / sqrtf(float(d.d));
 #define MF_STATS(T, DD)                                                                  \
   k_stats_simt<T, DD><<<grid, d.B, 0, st>>>(                                             \
       static_cast<const T*>(Q), static_cast<const T*>(K), d.cu_seqlens, m.cu_qb, m.cu_blk, \
-      d.nseq, d.Hs, d.B, scale, d.band_bias, d.band_width, sz.ntok, sz.nblocks, lse, part)
+      d.nseq, d.Hs, d.B, scale, d.band_bias, d.band_width, sz.ntok, sz.nblocks, r.qb_lo, lse, \
+      part)
   if (d.dt == MF_F32) {
     if (d.d == 64) MF_STATS(float, 64); else MF_STATS(float, 128);
   } else {
@@ -175,10 +185,10 @@ cudaError_t launch_stats_simt(const mf_attn_desc& d, const Sizes& sz, const Meta
   return cudaGetLastError();
 }
 
-// mass[b] = sum_h part[h][b], float64 in head order.
+// mass[b] = sum_h part[h][b], float64 in head order, for b in [blk_lo, blk_hi).
 __global__ void k_mass_reduce(const float* __restrict__ part, int Hs, int64_t nblocks,
-                              float* __restrict__ mass) {
-  for (int64_t b = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; b < nblocks;
+                              int64_t blk_lo, int64_t blk_hi, float* __restrict__ mass) {
+  for (int64_t b = blk_lo + blockIdx.x * int64_t(blockDim.x) + threadIdx.x; b < blk_hi;
        b += int64_t(gridDim.x) * blockDim.x) {
     double t = 0.0;
     for (int h = 0; h < Hs; ++h) t += double(part[int64_t(h) * nblocks + b]);
@@ -186,11 +196,11 @@ __global__ void k_mass_reduce(const float* __restrict__ part, int Hs, int64_t nb
   }
 }
 
-cudaError_t launch_mass_reduce(const float* part, int Hs, int64_t nblocks, float* mass,
-                               cudaStream_t st) {
-  int grid = int(std::min<int64_t>((nblocks + 255) / 256, 148 * 8));
-  if (grid < 1) grid = 1;
-  k_mass_reduce<<<grid, 256, 0, st>>>(part, Hs, nblocks, mass);
+cudaError_t launch_mass_reduce(const float* part, int Hs, int64_t nblocks, int64_t blk_lo,
+                               int64_t blk_hi, float* mass, cudaStream_t st) {
+  if (blk_hi <= blk_lo) return cudaSuccess;
+  int grid = int(std::min<int64_t>((blk_hi - blk_lo + 255) / 256, 148 * 8));
+  k_mass_reduce<<<grid, 256, 0, st>>>(part, Hs, nblocks, blk_lo, blk_hi, mass);
   return cudaGetLastError();
 }
 
@@ -202,9 +212,10 @@ __global__ void __launch_bounds__(128) k_extract_simt(
     const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ qb_seq,
     const int32_t* __restrict__ qb_idx, const int64_t* __restrict__ row_ptr,
     const int32_t* __restrict__ col_idx, int64_t capacity, int Hs, int B, float scale,
-    float band_bias, int band_width, int64_t ntok, T* __restrict__ values) {
+    float band_bias, int band_width, int64_t ntok, int64_t qb_lo, T* __restrict__ values) {
   __shared__ float ks[kKeyTile][D + 1];
-  const int gqb = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int64_t gqb = qb_lo + blockIdx.x;
+  const int h = blockIdx.y, tid = threadIdx.x;
   const int s = qb_seq[gqb], qb = qb_idx[gqb];
   const int seq0 = cu_seqlens[s];
   const int L = cu_seqlens[s + 1] - seq0;
@@ -241,16 +252,17 @@ __global__ void __launch_bounds__(128) k_extract_simt(
   }
 }
 
-cudaError_t launch_extract_simt(const mf_attn_desc& d, const Sizes& sz, const void* Q,
-                                const void* K, const float* lse, const mf_csr_cache& c,
-                                cudaStream_t st) {
-  dim3 grid(unsigned(sz.nqb), unsigned(d.Hs));
+cudaError_t launch_extract_simt(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                                const void* Q, const void* K, const float* lse,
+                                const mf_csr_cache& c, cudaStream_t st) {
+  if (r.qb_hi <= r.qb_lo) return cudaSuccess;
+  dim3 grid(unsigned(r.qb_hi - r.qb_lo), unsigned(d.Hs));
   const float scale = 1.0f / sqrtf(float(d.d));
 #define MF_EXTRACT(T, DD)                                                                 \
   k_extract_simt<T, DD><<<grid, d.B, 0, st>>>(                                            \
       static_cast<const T*>(Q), static_cast<const T*>(K), lse, d.cu_seqlens, c.qb_seq,    \
       c.qb_idx, c.row_ptr, c.col_idx, c.nnz_capacity, d.Hs, d.B, scale, d.band_bias,      \
-      d.band_width, sz.ntok, static_cast<T*>(c.values))
+      d.band_width, sz.ntok, r.qb_lo, static_cast<T*>(c.values))
   if (d.dt == MF_F32) {
     if (d.d == 64) MF_EXTRACT(float, 64); else MF_EXTRACT(float, 128);
   } else {

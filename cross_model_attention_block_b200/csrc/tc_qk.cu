@@ -92,6 +92,7 @@ struct Params {
   float* part;             // stats: out [Hs][nblocks]
   const int32_t* slot;     // extract: block -> cache entry or -1
   __nv_bfloat16* values;   // extract: out
+  int64_t qb_lo, qb_hi;    // global query blocks whose rows and blocks are written
   unsigned* status;
 };
 
@@ -192,12 +193,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.drain, 1);
     fence_barrier_init();
   }
+  // global index of this sequence's query block 0; a query block outside
+  // [qb_lo, qb_hi) is computed with its tile but nothing of it is written
+  const int64_t gq0 = p.cu_qb[s];
+  auto in_range = [&](int qb) { return gq0 + qb >= p.qb_lo && gq0 + qb < p.qb_hi; };
   if (MODE == kExtract) {
     const int64_t cb = p.cu_blk[s];
     for (int i = threadIdx.x; i < 2 * kMaxBlocksPerSeq; i += kThreads) {
       const int a = i / kMaxBlocksPerSeq, kb = i % kMaxBlocksPerSeq;
       const int qb = (BB == 128) ? (a == 0 ? t : -1) : 2 * t + a;
-      sm.slots[a][kb] = (qb >= 0 && qb < nqb_s && kb <= qb)
+      sm.slots[a][kb] = (qb >= 0 && qb < nqb_s && kb <= qb && in_range(qb))
                             ? p.slot[cb + int64_t(qb) * (qb + 1) / 2 + kb]
                             : -1;
     }
@@ -440,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l = l_run * ex2(m_run - Mu) + o.y * ex2(o.x - Mu);
         lse2 = valid ? M + lg2(l) : 0.f;
       }
-      if (valid && wg == 0) p.lse[int64_t(h) * p.ntok + seq0 + ri] = lse2 * kLn2;
+      if (valid && wg == 0 && in_range(ri / BB)) p.lse[int64_t(h) * p.ntok + seq0 + ri] = lse2 * kLn2;
       tmem_wait_st();
       tc_fence_before();
       named_sync_epilogue();  // both groups' log partials are in TMEM
@@ -464,13 +469,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (BB == 128) {
             const float m = (sm.red[wg][0][lane] + sm.red[wg][1][lane]) +
                             (sm.red[wg][2][lane] + sm.red[wg][3][lane]);
-            if (kb <= t) p.part[int64_t(h) * p.nblocks + cb + int64_t(t) * (t + 1) / 2 + kb] = m;
+            if (kb <= t && in_range(t))
+              p.part[int64_t(h) * p.nblocks + cb + int64_t(t) * (t + 1) / 2 + kb] = m;
           } else {
             const int qa = 2 * t, qbb = 2 * t + 1;
             const float m0 = sm.red[wg][0][lane] + sm.red[wg][1][lane];
             const float m1 = sm.red[wg][2][lane] + sm.red[wg][3][lane];
-            if (kb <= qa) p.part[int64_t(h) * p.nblocks + cb + int64_t(qa) * (qa + 1) / 2 + kb] = m0;
-            if (qbb < nqb_s && kb <= qbb)
+            if (kb <= qa && in_range(qa))
+              p.part[int64_t(h) * p.nblocks + cb + int64_t(qa) * (qa + 1) / 2 + kb] = m0;
+            if (qbb < nqb_s && kb <= qbb && in_range(qbb))
               p.part[int64_t(h) * p.nblocks + cb + int64_t(qbb) * (qbb + 1) / 2 + kb] = m1;
           }
         }
@@ -563,11 +570,11 @@ cudaError_t make_tmap_bf16(CUtensorMap* m, const void* base, int rank, const uin
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                             const void* Q, const void* K, float* lse, float* part,
-                             const int32_t* slot, void* values, int64_t capacity,
+static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                             const Meta& m, const void* Q, const void* K, float* lse,
+                             float* part, const int32_t* slot, void* values, int64_t capacity,
                              cudaStream_t st) {
-  if (sz.ntiles == 0) return cudaSuccess;
+  if (r.ntiles == 0) return cudaSuccess;
   CUtensorMap tq, tk;
   const uint64_t cols = uint64_t(d.Hs) * d.d;
   cudaError_t e = make_tmap_2d_bf16(&tq, Q, uint64_t(sz.ntok), cols, 64, qk::kTile, true);
@@ -593,7 +600,7 @@ static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, c
   p.tiles = m.tiles;
   p.cu_blk = m.cu_blk;
   p.cu_qb = m.cu_qb;
-  p.ntiles = int(sz.ntiles);
+  p.ntiles = int(r.ntiles);
   p.Hs = d.Hs;
   p.B = d.B;
   p.band_width = d.band_width;
@@ -605,9 +612,11 @@ static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, c
   p.part = part;
   p.slot = slot;
   p.values = static_cast<__nv_bfloat16*>(values);
+  p.qb_lo = r.qb_lo;
+  p.qb_hi = r.qb_hi;
   p.status = status_word();
   const size_t smem = sizeof(qk::Smem) + 1024;
-  const unsigned grid = unsigned(sz.ntiles) * unsigned(d.Hs);
+  const unsigned grid = unsigned(r.ntiles) * unsigned(d.Hs);
 #define MF_QK(MODE, BB)                                                                       \
   do {                                                                                        \
     e = cudaFuncSetAttribute(qk::k_qk<MODE, BB>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
@@ -624,17 +633,17 @@ static cudaError_t launch_qk(int mode, const mf_attn_desc& d, const Sizes& sz, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_stats_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                            const void* Q, const void* K, float* lse, float* part,
-                            cudaStream_t st) {
-  return launch_qk(qk::kStats, d, sz, m, Q, K, lse, part, nullptr, nullptr, 0, st);
+cudaError_t launch_stats_tc(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                            const Meta& m, const void* Q, const void* K, float* lse,
+                            float* part, cudaStream_t st) {
+  return launch_qk(qk::kStats, d, sz, r, m, Q, K, lse, part, nullptr, nullptr, 0, st);
 }
 
-cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
-                              const void* Q, const void* K, const float* lse,
+cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
+                              const Meta& m, const void* Q, const void* K, const float* lse,
                               const int32_t* slot, void* values, int64_t capacity,
                               cudaStream_t st) {
-  return launch_qk(qk::kExtract, d, sz, m, Q, K, const_cast<float*>(lse), nullptr, slot,
+  return launch_qk(qk::kExtract, d, sz, r, m, Q, K, const_cast<float*>(lse), nullptr, slot,
                    values, capacity, st);
 }
 

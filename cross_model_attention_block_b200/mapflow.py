@@ -25,7 +25,8 @@ MF_BF16, MF_F32 = 0, 1
 
 EXPORTED = [
     "mf_version", "mf_last_error", "mf_layout_sizes", "mf_block_stats_workspace",
-    "mf_block_stats", "mf_select_extract_workspace", "mf_select_extract",
+    "mf_block_stats", "mf_block_stats_range", "mf_select_extract_workspace",
+    "mf_select_extract", "mf_select_extract_range",
     "mf_mapped_av_workspace", "mf_mapped_av", "mf_mapped_av_range", "mf_block_stats_noalloc",
     "mf_block_stats_noalloc_max_workspace",
     "mf_mapped_av_plan", "mf_path_info", "mf_exp2_fma_eval", "mf_selftest_timeout", "mf_sync_status", "mf_prefix_hash",
@@ -81,8 +82,11 @@ def load_library(path: str = LIB_PATH):
         "mf_layout_sizes": (C.c_int, [I32, P, I32, P, P]),
         "mf_block_stats_workspace": (SZ, [P]),
         "mf_block_stats": (C.c_int, [P, P, P, P, P, P, SZ, P]),
+        "mf_block_stats_range": (C.c_int, [P, P, P, P, P, I64, I64, P, SZ, P]),
         "mf_select_extract_workspace": (SZ, [P]),
         "mf_select_extract": (C.c_int, [P, P, P, P, P, C.c_double, P, P, SZ, P]),
+        "mf_select_extract_range": (C.c_int, [P, P, P, P, P, C.c_double, P, I64, I64, P, SZ,
+                                              P]),
         "mf_mapped_av_workspace": (SZ, [P, P, I32, P]),
         "mf_mapped_av": (C.c_int, [P, P, I32, P, P, P, P, SZ, P]),
         "mf_mapped_av_range": (C.c_int, [P, P, I32, P, P, P, I64, I64, P, SZ, P]),
@@ -172,6 +176,19 @@ class Context:
     def layout_sizes(self):
         return layout_sizes(self.cu_seqlens_host, self.B)
 
+    def range_blocks(self, qb_begin, qb_end):
+        """Causal blocks of the global query blocks [qb_begin, qb_end): the
+        CSR capacity a cache of that range can never overflow."""
+        n = 0
+        q0 = 0
+        for L in np.diff(self.cu_seqlens_host):
+            nq = (int(L) + self.B - 1) // self.B
+            a, b = max(qb_begin - q0, 0), min(qb_end - q0, nq)
+            if a < b:
+                n += b * (b + 1) // 2 - a * (a + 1) // 2
+            q0 += nq
+        return n
+
 
 def layout_sizes(cu_seqlens_host, B):
     """(nqb_total, nblocks_total) of a context."""
@@ -182,8 +199,10 @@ def layout_sizes(cu_seqlens_host, B):
     return a.value, b.value
 
 
-def block_stats(ctx: Context, Q, K, lse=None, mass=None):
-    """Stage 1: lse [Hs, ntok] float32 and block masses [nblocks] float32."""
+def block_stats(ctx: Context, Q, K, lse=None, mass=None, qb_range=None):
+    """Stage 1: lse [Hs, ntok] float32 and block masses [nblocks] float32.
+    `qb_range` = (begin, end) restricts the call to those global query
+    blocks: only their lse rows and block masses are written."""
     L = load_library()
     d = ctx.desc()
     _, nblocks = ctx.layout_sizes()
@@ -196,8 +215,14 @@ def block_stats(ctx: Context, Q, K, lse=None, mass=None):
     if nbytes == 0:
         _check(MF_ERR_INVALID_ARG)
     ws, wsp = _workspace(nbytes, dev)
-    _check(L.mf_block_stats(C.byref(d), _ptr(Q), _ptr(K), _ptr(lse), _ptr(mass),
-                            C.c_void_p(wsp), nbytes, _stream()))
+    if qb_range is None:
+        _check(L.mf_block_stats(C.byref(d), _ptr(Q), _ptr(K), _ptr(lse), _ptr(mass),
+                                C.c_void_p(wsp), nbytes, _stream()))
+    else:
+        _check(L.mf_block_stats_range(C.byref(d), _ptr(Q), _ptr(K), _ptr(lse), _ptr(mass),
+                                      int(qb_range[0]), int(qb_range[1]), C.c_void_p(wsp),
+                                      nbytes, _stream()))
+    ctx._stats_ws = ws  # keep the workspace alive until the stream has used it
     return lse, mass
 
 
@@ -236,8 +261,11 @@ class Cache:
             self.capacity, B // 16, B // 8, 2, Hs, 8, 8)
 
 
-def select_extract(ctx: Context, Q, K, lse, mass, tau, cache: Cache | None = None):
-    """Stage 2: kept blocks per query block (CSR) and their probability blocks."""
+def select_extract(ctx: Context, Q, K, lse, mass, tau, cache: Cache | None = None,
+                   qb_range=None):
+    """Stage 2: kept blocks per query block (CSR) and their probability blocks.
+    `qb_range` = (begin, end) restricts the call to those global query blocks;
+    the CSR rows of every other query block are empty."""
     L = load_library()
     d = ctx.desc()
     if cache is None:
@@ -247,8 +275,14 @@ def select_extract(ctx: Context, Q, K, lse, mass, tau, cache: Cache | None = Non
     if nbytes == 0:
         _check(MF_ERR_INVALID_ARG)
     ws, wsp = _workspace(nbytes, Q.device)
-    _check(L.mf_select_extract(C.byref(d), _ptr(Q), _ptr(K), _ptr(lse), _ptr(mass),
-                               float(tau), C.byref(cs), C.c_void_p(wsp), nbytes, _stream()))
+    if qb_range is None:
+        _check(L.mf_select_extract(C.byref(d), _ptr(Q), _ptr(K), _ptr(lse), _ptr(mass),
+                                   float(tau), C.byref(cs), C.c_void_p(wsp), nbytes, _stream()))
+    else:
+        _check(L.mf_select_extract_range(C.byref(d), _ptr(Q), _ptr(K), _ptr(lse), _ptr(mass),
+                                         float(tau), C.byref(cs), int(qb_range[0]),
+                                         int(qb_range[1]), C.c_void_p(wsp), nbytes,
+                                         _stream()))
     cache._ws = ws  # keep the workspace alive until the stream has used it
     return cache
 

@@ -149,6 +149,21 @@ mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
                          float* lse, float* mass, void* ws, size_t ws_bytes,
                          mf_stream_t stream);
 
+/* As mf_block_stats, restricted to the global query blocks [qb_begin,
+ * qb_end) (global order: sequence by sequence): only the lse rows of those
+ * query blocks and the masses of their blocks (a contiguous span of the mass
+ * array) are written; the rest of lse and mass is left as it was.  Every
+ * query block's statistics depend only on its own rows and the keys before
+ * them, so a context split into ranges -- one per GPU, or several per GPU --
+ * gives, entry for entry, the result of one call (article, first and third
+ * components: block statistics per position; chunked prefill).  Q and K must
+ * hold the whole context.  Arguments, workspace and errors as
+ * mf_block_stats, plus MF_ERR_INVALID_ARG unless
+ * 0 <= qb_begin <= qb_end <= nqb_total. */
+mf_status mf_block_stats_range(const mf_attn_desc* desc, const void* Q, const void* K,
+                               float* lse, float* mass, int64_t qb_begin, int64_t qb_end,
+                               void* ws, size_t ws_bytes, mf_stream_t stream);
+
 /* Block statistics without a caller workspace.  The article has no
  * counterpart: this exists for callers that cannot allocate device memory,
  * such as a serving engine that gave all free HBM to its KV-cache pool, or a
@@ -186,6 +201,21 @@ mf_status mf_select_extract(const mf_attn_desc* desc, const void* Q, const void*
                             const float* lse, const float* mass, double tau,
                             mf_csr_cache* out, void* ws, size_t ws_bytes,
                             mf_stream_t stream);
+
+/* As mf_select_extract, restricted to the global query blocks [qb_begin,
+ * qb_end): selection and extraction run on those query blocks only (lse and
+ * mass are read only there), and every other row of the CSR is left empty
+ * (row_ptr covers all nqb_total rows).  The kept sets and probability blocks
+ * of the range are those of one full call; the cache holds entries of the
+ * range only, so nnz_capacity can be the range's causal blocks.  A process
+ * that owns several ranges keeps one cache per range; mf_mapped_av_range over
+ * the same range reads it.  Arguments, workspace and errors as
+ * mf_select_extract, plus MF_ERR_INVALID_ARG unless
+ * 0 <= qb_begin <= qb_end <= nqb_total. */
+mf_status mf_select_extract_range(const mf_attn_desc* desc, const void* Q, const void* K,
+                                  const float* lse, const float* mass, double tau,
+                                  mf_csr_cache* out, int64_t qb_begin, int64_t qb_end,
+                                  void* ws, size_t ws_bytes, mf_stream_t stream);
 
 /* Stage 3, fused map-mix x V (article: the fused kernel reads the sparse
  * blocks, combines heads on chip and multiplies straight into the receiver's

@@ -252,3 +252,20 @@ def test_every_bf16_workload_runs_the_tensor_core_kernels(lib):
     assert mfb.path_info(odd, 24, 8)["mapped_av_tc"] is False      # Hr not 16 or 32
     with pytest.raises(mfb.MapflowError):
         mfb.path_info(odd, 30, 8)                                  # Hr not a multiple of Hkv
+
+
+def test_range_forms_reject_bad_ranges_before_any_launch(lib):
+    """The statistics and selection range forms check the range on the host."""
+    import ctypes as C
+    ctx = mfb.Context.make([300, 200], 8, 128, 64, 2.0, 256, torch.bfloat16, device="cpu")
+    d = ctx.desc()
+    nqb, _ = ctx.layout_sizes()
+    for lo, hi in ((-1, 2), (3, 2), (0, nqb + 1)):
+        st = lib.mf_block_stats_range(C.byref(d), 16, 16, 16, 16, lo, hi, 256, 1 << 20, None)
+        assert st == mfb.MF_ERR_INVALID_ARG
+        assert "range" in lib.mf_last_error().decode()
+        cs = mfb.CsrCache(nqb, 10, 16, 16, 16, 16, 16, 8, 64, mfb.MF_BF16, 2, 16)
+        st = lib.mf_select_extract_range(C.byref(d), 16, 16, 16, 16, 0.9, C.byref(cs), lo, hi,
+                                         256, 1 << 20, None)
+        assert st == mfb.MF_ERR_INVALID_ARG
+        assert "range" in lib.mf_last_error().decode()

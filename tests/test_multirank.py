@@ -66,3 +66,25 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("RANK", "0")
     assert bench.main(["--impl", "reference", "--gpus", "2"]) == 0
     assert called == ["large_bf16_n32768"]
+
+
+def test_bench_rank_plans_cover_the_layer_once():
+    """bench.py --gpus N: the ranks' query-block ranges cover every query block
+    of the layer exactly once (one sequence: zig-zag pairs; varlen batch:
+    whole sequences), and their rows and causal pairs add up to the layer's."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from cross_model_attention_block_b200 import synth
+    for name in ("large_bf16_n32768", "mid_bf16_n8192", "varlen_paged_64seq"):
+        wl = synth.workloads()[name]
+        nqb = sum((L + wl.B - 1) // wl.B for L in wl.lengths)
+        full_rows, full_pairs = bench.plan_units(wl, [(0, nqb)])
+        assert full_rows == wl.ntok
+        assert full_pairs == sum(L * (L + 1) // 2 for L in wl.lengths)
+        for world in (1, 2, 4, 8):
+            plans = [bench.rank_plan(wl, r, world) for r in range(world)]
+            blocks = sorted(g for p in plans for a, b in p for g in range(a, b))
+            assert blocks == list(range(nqb)), (name, world)
+            units = [bench.plan_units(wl, p) for p in plans]
+            assert sum(u[0] for u in units) == full_rows
+            assert sum(u[1] for u in units) == full_pairs

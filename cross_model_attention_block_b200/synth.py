@@ -18,6 +18,9 @@ datasets; these seeded generators stand in for them:
   workload dtype by round-to-nearest-even.
 * Varlen batches draw log-uniform lengths and a random page permutation from
   their own stream.
+* Multi-turn contexts (the Round Attention page's conversations) draw round
+  lengths in whole blocks, uniform in [2, 16] blocks, from their own stream
+  (seed 3) until the sequence is covered; the last round is cut to fit.
 """
 from __future__ import annotations
 
@@ -53,6 +56,10 @@ class Workload:
     sender_layers: int = 1
     # receivers: list of (name, n_layers, layer_table)
     receivers: list = field(default_factory=list)
+    # multi-turn contexts: round start offsets per sequence (token offsets
+    # within the sequence, then its length), and the watershed sender layer
+    rounds: list = field(default_factory=list)
+    watershed: int = 0
 
     @property
     def ntok(self) -> int:
@@ -89,12 +96,27 @@ def workloads() -> dict:
         "multi_receiver_n16384", [16384], Hs=40, Hr=32, Hkv=8, d=128, B=64,
         tau=0.9, band_bias=2.0, band_width=256, dtype="bf16", seed=0,
         sender_layers=8, receivers=[("r1", 6, r1), ("r2", 4, r2)])
+    w["multi_turn_rounds_n8192"] = Workload(
+        "multi_turn_rounds_n8192", [8192], Hs=32, Hr=32, Hkv=8, d=128, B=64, tau=0.8,
+        band_bias=2.0, band_width=256, dtype="bf16", seed=0, sender_layers=4,
+        rounds=[round_starts(8192, 64, seed=3)], watershed=1)
     lens, _ = _varlen_lengths(64, 1024, 16384, seed=1)
     w["varlen_paged_64seq"] = Workload(
         "varlen_paged_64seq", lens, Hs=32, Hr=32, Hkv=8, d=128, B=64,
         tau=0.95, band_bias=2.0, band_width=256, dtype="bf16", seed=0,
         paged=True)
     return w
+
+
+def round_starts(L: int, B: int, seed: int, lo_blocks: int = 2, hi_blocks: int = 16):
+    """Round start offsets of one sequence of L tokens, then L: each round a
+    whole number of blocks drawn uniformly in [lo_blocks, hi_blocks]."""
+    rng = np.random.default_rng(seed)
+    starts = [0]
+    while starts[-1] < L:
+        n = int(rng.integers(lo_blocks, hi_blocks + 1))
+        starts.append(min(L, starts[-1] + n * B))
+    return starts
 
 
 def cu_seqlens(lengths) -> np.ndarray:

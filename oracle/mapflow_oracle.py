@@ -28,9 +28,22 @@ block; band bias beta added to the scaled logit when 0 <= i - j < band_width;
 contiguous GQA grouping g(r) = floor(r * Hkv / Hr); blocks aligned to each
 sequence start, no attention across sequences, partial last blocks.
 
+Round-level selection (the Round Attention page, "方法详解": a watershed
+layer's attention decides, per conversation round, which earlier rounds to
+keep; the kept rounds then serve the later layers) is the second selection
+policy over the same block cache.  Readings: every round starts on a block
+boundary of its sequence; a query round always keeps its own tokens and adds
+the fewest earlier rounds, heaviest first (ties to the lower round), whose
+mass together with its own reaches tau * T, where the mass of key round r for
+query round q sums P_h[i, j] over the heads, the rows i of q and the keys j
+of r (j <= i), and T sums it over every round up to q; tau >= 1 keeps every
+round.  One selection, taken at the watershed layer, gives the kept blocks of
+every later layer.
+
 Every function works on one sequence and one query block at a time, so memory
 stays O(B * L * Hs) and any single block can be checked at full size.
-Every function here is pinned by the tests in tests/test_oracle_pins.py.
+Every function here is pinned by the tests in tests/test_oracle_pins.py and
+tests/test_round_pins.py.
 """
 from __future__ import annotations
 
@@ -208,3 +221,86 @@ def run_layer(Q, K, V, W, lengths, Hkv: int, B: int, tau: float,
         res.append(r)
         start += L
     return res, O
+
+
+# ------------------------------------------------ round-level selection
+
+
+def round_of_token(round_starts, j: int) -> int:
+    """Index of the round holding token j (round_starts ascending, [0] = 0)."""
+    r = 0
+    while r + 1 < len(round_starts) and round_starts[r + 1] <= j:
+        r += 1
+    return r
+
+
+def round_mass(Qs, Ks, round_starts, q: int, band_bias: float, band_width: int,
+               rows_per_chunk: int = 64) -> np.ndarray:
+    """Attention mass of query round q on every round 0..q of one sequence.
+
+    m[r] = sum_h sum_{i in round q} sum_{j in round r, j <= i} P_h[i, j],
+    straight from the probabilities of the rows of round q (no block sums),
+    taken over the round's rows in chunks to bound memory.
+    round_starts: token offsets of the rounds, then the sequence length.
+    """
+    m = np.zeros(q + 1)
+    for c0 in range(round_starts[q], round_starts[q + 1], rows_per_chunk):
+        c1 = min(round_starts[q + 1], c0 + rows_per_chunk)
+        _, P = lse_and_probs(scores(Qs, Ks, c0, c1, band_bias, band_width))  # [Hs, rows, c1]
+        for r in range(q + 1):
+            m[r] += P[:, :, round_starts[r]:min(round_starts[r + 1], c1)].sum()
+    return m
+
+
+def select_rounds(m: np.ndarray, tau: float) -> np.ndarray:
+    """Kept rounds of the query round q = len(m) - 1, ascending.
+
+    Round q is always kept.  Earlier rounds in order of mass descending, ties
+    to the lower index; keep the fewest k of them with m[q] + (sum of the
+    first k) >= tau * T, T = sum(m) (fp64 sums in that order); all of them if
+    never reached; tau >= 1 keeps every round.
+    """
+    q = len(m) - 1
+    if tau >= 1.0:
+        return np.arange(q + 1)
+    T = float(np.sum(m))
+    order = sorted(range(q), key=lambda r: (-m[r], r))
+    c = float(m[q])
+    k = 0
+    while c < tau * T and k < q:
+        c += float(m[order[k]])
+        k += 1
+    return np.array(sorted(order[:k] + [q]), dtype=np.int64)
+
+
+def round_kept_blocks(kept_rounds, round_starts, qb: int, B: int) -> np.ndarray:
+    """Key blocks kb <= qb that lie in a kept round (rounds start on block
+    boundaries, so a block lies in exactly one round)."""
+    kept = set(int(r) for r in kept_rounds)
+    return np.array([kb for kb in range(qb + 1)
+                     if round_of_token(round_starts, kb * B) in kept], dtype=np.int64)
+
+
+def run_rounds_sequence(Qw, Kw, layers, W, Hkv: int, B: int, tau: float,
+                        round_starts, band_bias: float, band_width: int, qbs=None):
+    """Round selection on one sequence at the watershed layer (Qw, Kw), then
+    every layer of `layers` [(Q, K, V)] through its own probabilities on the
+    selected blocks.  Returns {qb: {"rounds": kept rounds of qb's round,
+    "kept": kept blocks, "O": [O of each layer]}}.
+    """
+    L = Qw.shape[0]
+    nqb = (L + B - 1) // B
+    kept_r = {}
+    out = {}
+    for qb in (range(nqb) if qbs is None else qbs):
+        q = round_of_token(round_starts, qb * B)
+        if q not in kept_r:
+            kept_r[q] = select_rounds(
+                round_mass(Qw, Kw, round_starts, q, band_bias, band_width), tau)
+        kept = round_kept_blocks(kept_r[q], round_starts, qb, B)
+        Os = []
+        for Q, K, V in layers:
+            _, P, _ = query_block(Q, K, qb, B, band_bias, band_width)
+            Os.append(mapped_av(mixed_map(P, kept, W, B), V, Hkv))
+        out[qb] = {"rounds": kept_r[q], "kept": kept, "O": Os}
+    return out

@@ -291,6 +291,61 @@ mf_status mf_select_extract_range(const mf_attn_desc* desc, const void* Q, const
   return MF_OK;
 }
 
+// ------------------------------------------------------- rounds, extraction
+
+// Checks a round layout against the context: starts ascending from 0 to ntok,
+// every non-empty sequence starts a round, every round starts on a block
+// boundary of its sequence and ends inside it.  *max_r: most rounds of one
+// sequence.
+static mf_status check_rounds(const mf_attn_desc& d, int32_t nrounds, const int32_t* st,
+                              int* max_r) {
+  if (nrounds < 1 || !st) return fail(MF_ERR_INVALID_ARG, "no rounds, or round_starts_host is NULL");
+  const int32_t* cu = d.cu_seqlens_host;
+  if (st[0] != 0 || st[nrounds] != cu[d.nseq])
+    return fail(MF_ERR_INVALID_ARG, "round starts must run from 0 to the token count");
+  int s = 0, in_seq = 0;
+  *max_r = 0;
+  for (int r = 0; r < nrounds; ++r) {
+    if (st[r + 1] <= st[r]) return fail(MF_ERR_INVALID_ARG, "round starts must increase");
+    while (s < d.nseq && cu[s + 1] <= st[r]) {
+      ++s;
+      in_seq = 0;
+    }
+    if (in_seq == 0 && st[r] != cu[s])
+      return fail(MF_ERR_INVALID_ARG, "a sequence does not start a round");
+    if ((st[r] - cu[s]) % d.B != 0)
+      return fail(MF_ERR_INVALID_ARG, "a round does not start on a block boundary");
+    if (st[r + 1] > cu[s + 1]) return fail(MF_ERR_INVALID_ARG, "a round crosses a sequence end");
+    *max_r = std::max(*max_r, ++in_seq);
+  }
+  return MF_OK;
+}
+
+static size_t rounds_ws(const mf_attn_desc& d, const Sizes& sz, int nrounds, int max_r,
+                        void* base, Meta* m, int32_t** r_seq, int32_t** r_first,
+                        uint8_t** flags, int32_t** counts) {
+  Carve c(base);
+  meta_bytes(c, d.nseq, sz.ntiles, m);
+  int32_t* a = c.take<int32_t>(size_t(nrounds));
+  int32_t* b = c.take<int32_t>(size_t(d.nseq) + 1);
+  uint8_t* f = c.take<uint8_t>(size_t(nrounds) * size_t(max_r));
+  int32_t* n = c.take<int32_t>(size_t(sz.nqb) + 1);
+  if (r_seq) *r_seq = a;
+  if (r_first) *r_first = b;
+  if (flags) *flags = f;
+  if (counts) *counts = n;
+  return c.used + 256;
+}
+
+static size_t extract_ws(const mf_attn_desc& d, const Sizes& sz, void* base, Meta* m,
+                         int32_t** slot) {
+  Carve c(base);
+  meta_bytes(c, d.nseq, sz.ntiles, m);
+  int32_t* s = c.take<int32_t>(size_t(sz.nblocks) + 1);
+  if (slot) *slot = s;
+  return c.used + 256;
+}
+
 static mf_status check_av(const mf_csr_cache* cache, const mf_attn_desc* desc, int32_t Hr,
                           const mf_v_desc* v, Sizes* sz) {
   mf_status st = check_desc(desc, sz);
@@ -357,6 +412,90 @@ mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc
                                            qb_begin, qb_end, s)
                      : launch_mapped_av_simt(*cache, d, sz, Hr, W, *v, O, qb_begin, qb_end, s);
   if (e != cudaSuccess) return cuda_fail(e, "mapped av");
+  return MF_OK;
+}
+
+size_t mf_select_rounds_workspace(const mf_attn_desc* desc, int32_t nrounds,
+                                  const int32_t* round_starts_host) {
+  Sizes sz;
+  if (check_desc(desc, &sz) != MF_OK) return 0;
+  int max_r = 0;
+  if (check_rounds(*desc, nrounds, round_starts_host, &max_r) != MF_OK) return 0;
+  return rounds_ws(*desc, sz, nrounds, max_r, nullptr, nullptr, nullptr, nullptr, nullptr,
+                   nullptr);
+}
+
+mf_status mf_select_rounds(const mf_attn_desc* desc, const float* mass, int32_t nrounds,
+                           const int32_t* round_starts, const int32_t* round_starts_host,
+                           double tau, mf_csr_cache* out, void* ws, size_t ws_bytes,
+                           mf_stream_t stream) {
+  Sizes sz;
+  mf_status st = check_desc(desc, &sz);
+  if (st != MF_OK) return st;
+  const mf_attn_desc& d = *desc;
+  if (!mass || !round_starts) return fail(MF_ERR_INVALID_ARG, "mass or round_starts is NULL");
+  if (!(tau > 0.0) || !std::isfinite(tau)) return fail(MF_ERR_INVALID_ARG, "tau must be > 0");
+  int max_r = 0;
+  st = check_rounds(d, nrounds, round_starts_host, &max_r);
+  if (st != MF_OK) return st;
+  st = check_cache(out, d, sz);
+  if (st != MF_OK) return st;
+  const size_t need = rounds_ws(d, sz, nrounds, max_r, nullptr, nullptr, nullptr, nullptr,
+                                nullptr, nullptr);
+  if (!ws || !aligned256(ws) || ws_bytes < need)
+    return fail(MF_ERR_WORKSPACE, "workspace missing, not 256-byte aligned or too small");
+  if (!status_word()) return fail(MF_ERR_CUDA, "no CUDA device");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Meta m;
+  int32_t *r_seq = nullptr, *r_first = nullptr, *counts = nullptr;
+  uint8_t* flags = nullptr;
+  rounds_ws(d, sz, nrounds, max_r, ws, &m, &r_seq, &r_first, &flags, &counts);
+  cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, 0, sz.nqb, m, s);
+  if (e != cudaSuccess) return cuda_fail(e, "meta");
+  if (sz.nqb == 0) {
+    e = cudaMemsetAsync(out->row_ptr, 0, sizeof(int64_t), s);
+    return e == cudaSuccess ? MF_OK : cuda_fail(e, "row_ptr");
+  }
+  e = launch_select_rounds(d, sz, m, mass, nrounds, round_starts, max_r, tau, *out, r_seq,
+                           r_first, flags, counts, s);
+  if (e != cudaSuccess) return cuda_fail(e, "select rounds");
+  return MF_OK;
+}
+
+size_t mf_extract_workspace(const mf_attn_desc* desc) {
+  Sizes sz;
+  if (check_desc(desc, &sz) != MF_OK) return 0;
+  return extract_ws(*desc, sz, nullptr, nullptr, nullptr);
+}
+
+mf_status mf_extract(const mf_attn_desc* desc, const void* Q, const void* K, const float* lse,
+                     const mf_csr_cache* cache, void* ws, size_t ws_bytes, mf_stream_t stream) {
+  Sizes sz;
+  mf_status st = check_desc(desc, &sz);
+  if (st != MF_OK) return st;
+  const mf_attn_desc& d = *desc;
+  if (!Q || !K || !lse) return fail(MF_ERR_INVALID_ARG, "Q, K or lse is NULL");
+  st = check_cache(cache, d, sz);
+  if (st != MF_OK) return st;
+  if (!ws || !aligned256(ws) || ws_bytes < extract_ws(d, sz, nullptr, nullptr, nullptr))
+    return fail(MF_ERR_WORKSPACE, "workspace missing, not 256-byte aligned or too small");
+  if (!status_word()) return fail(MF_ERR_CUDA, "no CUDA device");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Meta m;
+  int32_t* slot = nullptr;
+  extract_ws(d, sz, ws, &m, &slot);
+  const QbRange r = range_of(d, sz, 0, sz.nqb);
+  cudaError_t e = launch_meta(d.nseq, d.cu_seqlens, d.B, r.qb_lo, r.qb_hi, m, s);
+  if (e != cudaSuccess) return cuda_fail(e, "meta");
+  if (sz.nqb == 0) return MF_OK;
+  if (use_tc(d)) {
+    e = launch_csr_slots(sz, m, *cache, slot, s);
+    if (e != cudaSuccess) return cuda_fail(e, "csr slots");
+    e = launch_extract_tc(d, sz, r, m, Q, K, lse, slot, cache->values, cache->nnz_capacity, s);
+  } else {
+    e = launch_extract_simt(d, sz, r, Q, K, lse, *cache, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "extract");
   return MF_OK;
 }
 

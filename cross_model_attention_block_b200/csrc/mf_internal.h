@@ -107,6 +107,23 @@ cudaError_t launch_select(const mf_attn_desc& d, const Sizes& sz, const QbRange&
                           const Meta& m, const float* mass, double tau, const mf_csr_cache& c,
                           int32_t* counts, uint8_t* keep, int32_t* slot, cudaStream_t st);
 
+// Global query block -> (sequence, index) map; exclusive int64 scan of counts.
+void launch_qb_map(int64_t nqb, int nseq, const int32_t* cu_qb, int32_t* qb_seq,
+                   int32_t* qb_idx, int grid, cudaStream_t st);
+void launch_scan(const int32_t* counts, int64_t n, int64_t* row_ptr, cudaStream_t st);
+
+// Round-level selection: CSR rows of every query block from the kept rounds
+// of its query round (r_seq [nrounds], r_first [nseq+1], flags
+// [nrounds][max_r], counts [nqb] are workspace).
+cudaError_t launch_select_rounds(const mf_attn_desc& d, const Sizes& sz, const Meta& m,
+                                 const float* mass, int nrounds, const int32_t* starts,
+                                 int max_r, double tau, const mf_csr_cache& c,
+                                 int32_t* r_seq, int32_t* r_first, uint8_t* flags,
+                                 int32_t* counts, cudaStream_t st);
+// Block -> entry map of a filled CSR (slot [nblocks], -1 where not kept).
+cudaError_t launch_csr_slots(const Sizes& sz, const Meta& m, const mf_csr_cache& c,
+                             int32_t* slot, cudaStream_t st);
+
 cudaError_t launch_extract_simt(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
                                 const void* Q, const void* K, const float* lse,
                                 const mf_csr_cache& c, cudaStream_t st);

@@ -139,6 +139,15 @@ __global__ void k_fill(const int64_t* __restrict__ row_ptr, const uint8_t* __res
   if (over) atomicOr(status, kStatusCapacity);
 }
 
+void launch_qb_map(int64_t nqb, int nseq, const int32_t* cu_qb, int32_t* qb_seq,
+                   int32_t* qb_idx, int grid, cudaStream_t st) {
+  k_qb_map<<<grid, 256, 0, st>>>(nqb, nseq, cu_qb, qb_seq, qb_idx);
+}
+
+void launch_scan(const int32_t* counts, int64_t n, int64_t* row_ptr, cudaStream_t st) {
+  k_scan<<<1, 1024, 0, st>>>(counts, n, row_ptr);
+}
+
 cudaError_t launch_select(const mf_attn_desc& d, const Sizes& sz, const QbRange& r,
                           const Meta& m, const float* mass, double tau, const mf_csr_cache& c,
                           int32_t* counts, uint8_t* keep, int32_t* slot, cudaStream_t st) {

@@ -17,7 +17,8 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmapflow.so")
+# the in-tree build; MAPFLOW_LIB names another build of the same library
+LIB_PATH = os.environ.get("MAPFLOW_LIB") or os.path.join(_HERE, "libmapflow.so")
 
 MF_OK, MF_ERR_INVALID_ARG, MF_ERR_UNSUPPORTED, MF_ERR_WORKSPACE = 0, 1, 2, 3
 MF_ERR_CUDA, MF_ERR_TIMEOUT, MF_ERR_NOT_FOUND, MF_ERR_CAPACITY = 4, 5, 6, 7
@@ -26,7 +27,8 @@ MF_BF16, MF_F32 = 0, 1
 EXPORTED = [
     "mf_version", "mf_last_error", "mf_layout_sizes", "mf_block_stats_workspace",
     "mf_block_stats", "mf_block_stats_range", "mf_select_extract_workspace",
-    "mf_select_extract", "mf_select_extract_range",
+    "mf_select_extract", "mf_select_extract_range", "mf_extract_workspace", "mf_extract",
+    "mf_select_rounds_workspace", "mf_select_rounds", "mf_cache_offload", "mf_cache_fetch",
     "mf_mapped_av_workspace", "mf_mapped_av", "mf_mapped_av_range", "mf_block_stats_noalloc",
     "mf_block_stats_noalloc_max_workspace",
     "mf_mapped_av_plan", "mf_path_info", "mf_exp2_fma_eval", "mf_selftest_timeout", "mf_sync_status", "mf_prefix_hash",
@@ -87,6 +89,12 @@ def load_library(path: str = LIB_PATH):
         "mf_select_extract": (C.c_int, [P, P, P, P, P, C.c_double, P, P, SZ, P]),
         "mf_select_extract_range": (C.c_int, [P, P, P, P, P, C.c_double, P, I64, I64, P, SZ,
                                               P]),
+        "mf_extract_workspace": (SZ, [P]),
+        "mf_extract": (C.c_int, [P, P, P, P, P, P, SZ, P]),
+        "mf_select_rounds_workspace": (SZ, [P, I32, P]),
+        "mf_select_rounds": (C.c_int, [P, P, I32, P, P, C.c_double, P, P, SZ, P]),
+        "mf_cache_offload": (C.c_int, [P, P, P]),
+        "mf_cache_fetch": (C.c_int, [P, P, I64, I64, P]),
         "mf_mapped_av_workspace": (SZ, [P, P, I32, P]),
         "mf_mapped_av": (C.c_int, [P, P, I32, P, P, P, P, SZ, P]),
         "mf_mapped_av_range": (C.c_int, [P, P, I32, P, P, P, I64, I64, P, SZ, P]),
@@ -118,6 +126,10 @@ def _check(status):
 
 
 def _stream():
+    # without a CUDA device only the library's argument checks can run (they
+    # return before anything is enqueued); NULL then stands for the stream
+    if not torch.cuda.is_available():
+        return C.c_void_p(None)
     return C.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
@@ -227,9 +239,10 @@ def block_stats(ctx: Context, Q, K, lse=None, mass=None, qb_range=None):
 
 
 class Cache:
-    """Caller-owned device buffers of one CSR block cache."""
+    """Caller-owned buffers of one CSR block cache (device memory, or pinned
+    host memory for the host tier)."""
 
-    def __init__(self, ctx: Context, capacity=None, device="cuda"):
+    def __init__(self, ctx: Context, capacity=None, device="cuda", pin=False):
         nqb, nblocks = ctx.layout_sizes()
         cap = nblocks if capacity is None else int(capacity)
         self.ctx = ctx
@@ -241,6 +254,9 @@ class Cache:
         self.qb_idx = torch.empty(max(nqb, 1), dtype=torch.int32, device=device)
         nvals = max(cap, 1) * ctx.B * ctx.B * ctx.Hs
         self.values = torch.empty(nvals, dtype=ctx.dtype, device=device)
+        if pin:
+            for name in ("row_ptr", "col_idx", "qb_seq", "qb_idx", "values"):
+                setattr(self, name, getattr(self, name).pin_memory())
 
     def struct(self) -> CsrCache:
         return CsrCache(self.nqb, self.capacity, self.row_ptr.data_ptr(),
@@ -285,6 +301,62 @@ def select_extract(ctx: Context, Q, K, lse, mass, tau, cache: Cache | None = Non
                                          _stream()))
     cache._ws = ws  # keep the workspace alive until the stream has used it
     return cache
+
+
+def extract(ctx: Context, Q, K, lse, cache: Cache):
+    """Probability blocks of every entry of a filled CSR (this layer's Q, K, lse)."""
+    L = load_library()
+    d = ctx.desc()
+    nbytes = L.mf_extract_workspace(C.byref(d))
+    if nbytes == 0:
+        _check(MF_ERR_INVALID_ARG)
+    ws, wsp = _workspace(nbytes, Q.device)
+    cs = cache.struct()
+    _check(L.mf_extract(C.byref(d), _ptr(Q), _ptr(K), _ptr(lse), C.byref(cs), C.c_void_p(wsp),
+                        nbytes, _stream()))
+    cache._ws = ws
+    return cache
+
+
+def select_rounds(ctx: Context, mass, round_starts, tau, cache: Cache | None = None):
+    """Round-level selection from the watershed layer's block masses: the CSR
+    of every query block (values are written by `extract`, per layer).
+    round_starts: packed token offsets of the rounds, 0 .. ntok."""
+    L = load_library()
+    d = ctx.desc()
+    st = np.ascontiguousarray(round_starts, dtype=np.int32)
+    nr = len(st) - 1
+    dev = mass.device
+    st_dev = torch.from_numpy(st).to(dev)
+    if cache is None:
+        cache = Cache(ctx, device=dev)
+    nbytes = L.mf_select_rounds_workspace(C.byref(d), nr, st.ctypes.data)
+    if nbytes == 0:
+        _check(L.mf_select_rounds(C.byref(d), _ptr(mass), nr, _ptr(st_dev), st.ctypes.data,
+                                  float(tau), None, None, 0, _stream()))
+        _check(MF_ERR_INVALID_ARG)
+    ws, wsp = _workspace(nbytes, dev)
+    cs = cache.struct()
+    _check(L.mf_select_rounds(C.byref(d), _ptr(mass), nr, _ptr(st_dev), st.ctypes.data,
+                              float(tau), C.byref(cs), C.c_void_p(wsp), nbytes, _stream()))
+    cache._round_ws = (ws, st_dev)
+    return cache
+
+
+def cache_offload(dev_cache: Cache, host_cache: Cache):
+    """Copy a device cache into a (pinned) host cache of the same layout."""
+    _check(load_library().mf_cache_offload(C.byref(dev_cache.struct()),
+                                           C.byref(host_cache.struct()), _stream()))
+    return host_cache
+
+
+def cache_fetch(host_cache: Cache, dev_cache: Cache, qb_range):
+    """Enqueue the copies of a range of rows of a host cache into a device
+    cache on the current stream."""
+    _check(load_library().mf_cache_fetch(C.byref(host_cache.struct()),
+                                         C.byref(dev_cache.struct()), int(qb_range[0]),
+                                         int(qb_range[1]), _stream()))
+    return dev_cache
 
 
 def mapped_av(cache: Cache, Hr, W, V, Hkv, page_table=None, page_size=16, O=None,

@@ -217,6 +217,48 @@ mf_status mf_select_extract_range(const mf_attn_desc* desc, const void* Q, const
                                   mf_csr_cache* out, int64_t qb_begin, int64_t qb_end,
                                   void* ws, size_t ws_bytes, mf_stream_t stream);
 
+/* Extraction for a given CSR: writes the probability blocks of every entry
+ * of `cache` (row_ptr, col_idx, qb_seq and qb_idx filled, e.g. by
+ * mf_select_extract of another layer or by mf_select_rounds) from this
+ * layer's Q, K and lse (article, first component: the kept blocks are
+ * extracted after the block statistics; Round Attention page, "方法详解": the
+ * rounds kept at the watershed layer serve the later layers).  Values as in
+ * mf_select_extract.  An entry whose key block is not a causal block of its
+ * query block is skipped and sets the device status (MF_ERR_INVALID_ARG via
+ * mf_sync_status).  Arguments and errors as mf_select_extract; the workspace
+ * is at least mf_extract_workspace(desc) bytes. */
+size_t mf_extract_workspace(const mf_attn_desc* desc);
+mf_status mf_extract(const mf_attn_desc* desc, const void* Q, const void* K, const float* lse,
+                     const mf_csr_cache* cache, void* ws, size_t ws_bytes, mf_stream_t stream);
+
+/* Round-level selection, a second selection policy over the same cache
+ * (Round Attention page, "方法详解": in a multi-turn context the attention
+ * of a watershed layer picks, for every conversation round, the earlier
+ * rounds that matter).  The context is split into nrounds rounds:
+ * round_starts [nrounds+1] int32 (device) and round_starts_host (host, the
+ * same values) are packed token offsets, from 0 to ntok; every non-empty
+ * sequence starts a round, every round starts on a block boundary of its
+ * sequence (offset from the sequence start a multiple of B) and ends inside
+ * it.  With mass the watershed layer's block masses (mf_block_stats), the
+ * mass of key round r for query round q is the float64 sum of the block
+ * masses of q's query blocks over r's key blocks (causal).  Query round q
+ * keeps its own round and the fewest earlier rounds, in order of mass
+ * descending with ties to the lower round, whose masses with its own reach
+ * tau * T (T: q's mass over rounds 0..q, float64); tau >= 1 keeps every
+ * round.  Every query block of q keeps the blocks of the kept rounds up to
+ * its own (ascending).  Fills row_ptr, col_idx, qb_seq, qb_idx of `out`;
+ * the values are written by mf_extract, once per layer that uses the
+ * selection.  Overflowing nnz_capacity sets the device status
+ * (MF_ERR_CAPACITY).  Errors: MF_ERR_INVALID_ARG (rounds that break the rules
+ * above, tau <= 0, NULL pointers), MF_ERR_WORKSPACE (workspace smaller than
+ * mf_select_rounds_workspace, which returns 0 for an invalid layout). */
+size_t mf_select_rounds_workspace(const mf_attn_desc* desc, int32_t nrounds,
+                                  const int32_t* round_starts_host);
+mf_status mf_select_rounds(const mf_attn_desc* desc, const float* mass, int32_t nrounds,
+                           const int32_t* round_starts, const int32_t* round_starts_host,
+                           double tau, mf_csr_cache* out, void* ws, size_t ws_bytes,
+                           mf_stream_t stream);
+
 /* Stage 3, fused map-mix x V (article: the fused kernel reads the sparse
  * blocks, combines heads on chip and multiplies straight into the receiver's
  * V, accumulating the output):
@@ -251,6 +293,34 @@ mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc
                              int32_t Hr, const void* W, const mf_v_desc* v, void* O,
                              int64_t qb_begin, int64_t qb_end, void* ws, size_t ws_bytes,
                              mf_stream_t stream);
+
+/* ---- host-memory tier of the cache (article, second component: the
+ * receiver's retrieval of cached blocks overlaps its recomputation of its
+ * first layers).  A cache that outlives the sender's request lives in host
+ * memory (pinned, for copies that overlap kernels); a receiver fetches the
+ * rows it needs into a device cache on a copy stream.  Both caches have the
+ * same layout (nqb_total, Hs, B, dt) and every entry sits at the same index
+ * in both, so a device cache filled range by range serves mf_mapped_av_range
+ * over each fetched range.  Only cudaMemcpyAsync is used; the library
+ * allocates nothing. */
+
+/* Copies a whole device cache (rows and entries row_ptr[nqb_total] of them)
+ * into host buffers.  Synchronizes `stream` first and reads the entry count
+ * with a blocking copy; the array copies are then enqueued on `stream`.
+ * Errors: MF_ERR_INVALID_ARG (layouts differ, NULL arrays), MF_ERR_CAPACITY
+ * (host capacity below the entry count), MF_ERR_CUDA. */
+mf_status mf_cache_offload(const mf_csr_cache* dev_src, mf_csr_cache* host_dst,
+                           mf_stream_t stream);
+
+/* Enqueues on `stream` the copies of the rows of global query blocks
+ * [qb_begin, qb_end) of a host cache into a device cache: row_ptr[qb_begin ..
+ * qb_end], qb_seq and qb_idx of those rows, and their entries (col_idx,
+ * values).  host_src's arrays are host memory (row_ptr is read on the host);
+ * dev_dst's are device memory.  Errors: MF_ERR_INVALID_ARG (layouts differ,
+ * a bad range, a device row_ptr in host_src), MF_ERR_CAPACITY (the rows'
+ * entries exceed dev_dst's capacity), MF_ERR_CUDA. */
+mf_status mf_cache_fetch(const mf_csr_cache* host_src, mf_csr_cache* dev_dst, int64_t qb_begin,
+                         int64_t qb_end, mf_stream_t stream);
 
 /* Diagnostic, not on the hot path: y[i] = 2^x[i] by the FMA-pipe
  * exponential written for the block-statistics epilogue (x = j + f,

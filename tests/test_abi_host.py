@@ -269,3 +269,50 @@ def test_range_forms_reject_bad_ranges_before_any_launch(lib):
                                          256, 1 << 20, None)
         assert st == mfb.MF_ERR_INVALID_ARG
         assert "range" in lib.mf_last_error().decode()
+
+
+@pytest.mark.parametrize("starts,msg", [
+    ([64, 128, 500], "from 0"),
+    ([0, 128, 128, 500], "increase"),
+    ([0, 100, 500], "block boundary"),
+    ([0, 128, 320, 500], "crosses"),
+    ([0, 128, 500], "crosses"),
+], ids=["not_from_zero", "not_increasing", "unaligned", "crosses_seq_end", "seq_without_round"])
+def test_round_layout_rejected_before_any_launch(lib, starts, msg):
+    """Rounds must run from 0 to ntok, start every sequence, start on block
+    boundaries of their sequence and end inside it (two sequences, 300 + 200
+    tokens, B = 64)."""
+    ctx = mfb.Context.make([300, 200], 8, 128, 64, 2.0, 256, torch.bfloat16, device="cpu")
+    mass = torch.zeros(ctx.layout_sizes()[1])
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.select_rounds(ctx, mass, starts, 0.9, cache=mfb.Cache(ctx, device="cpu"))
+    assert e.value.status == mfb.MF_ERR_INVALID_ARG
+    assert msg in str(e.value)
+
+
+def test_cache_tier_checks_layouts_and_ranges(lib):
+    """mf_cache_fetch / mf_cache_offload reject mismatched layouts and bad
+    ranges before any copy."""
+    ctx = mfb.Context.make([300], 8, 128, 64, 2.0, 256, torch.bfloat16, device="cpu")
+    a = mfb.Cache(ctx, device="cpu")
+    ctx2 = mfb.Context.make([300], 4, 128, 64, 2.0, 256, torch.bfloat16, device="cpu")
+    b = mfb.Cache(ctx2, device="cpu")
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.cache_fetch(a, b, (0, 1))
+    assert e.value.status == mfb.MF_ERR_INVALID_ARG and "differ" in str(e.value)
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.cache_offload(a, b)
+    assert e.value.status == mfb.MF_ERR_INVALID_ARG
+    with pytest.raises(mfb.MapflowError) as e:
+        mfb.cache_fetch(a, mfb.Cache(ctx, device="cpu"), (2, 99))
+    assert "range" in str(e.value)
+
+
+def test_overlap_chunk_ranges_cover_the_rows():
+    from cross_model_attention_block_b200 import overlap as ov
+    for nqb in (0, 1, 5, 128, 256):
+        for chunks in (1, 3, 8, 300):
+            r = ov.chunk_ranges(nqb, chunks)
+            covered = [g for a, b in r for g in range(a, b)]
+            assert covered == list(range(nqb))
+            assert all(a < b for a, b in r)

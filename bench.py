@@ -8,6 +8,7 @@ resident in HBM when the timed region starts; the kept map (tens of GB) is far
 larger than L2, so no separate L2 flush is done.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--mode path|rounds|overlap]
 
 With N > 1 (torchrun), the layer's query blocks are split across the ranks
 with no data-path collective (every query block's work is independent): a
@@ -16,6 +17,13 @@ sequences balanced by causal cost.  The total work is fixed as N grows
 (strong scaling); time = max over ranks.
 `--impl reference` times the CPU oracle on the host cores on a bounded
 sample of the same workload (rank 0 only).
+
+Two more measurements, one GPU each, print their own line:
+`--mode rounds` the round-level selection (multi-turn workload: selection at
+the watershed layer, then extraction and the fused kernel on every later
+layer); `--mode overlap` a receiver prefill that fetches a mapped layer's
+cache from pinned host memory while it recomputes its first layers, against
+the same calls issued serially.
 """
 from __future__ import annotations
 
@@ -425,19 +433,19 @@ def bench_ours(args, wl, rank, world, local_rank):
     stats_tf = alg["stats_flops"] / (t_stats * 1e-3) / 1e12
     ext_gbs = alg["extract_bytes"] / (t_sel * 1e-3) / 1e9
     hbm = peaks["hbm_gbs"]
-    # the kernels are timed inside a loop of back-to-back steps lasting about a
-    # second, so the tensor denominator is the sustained cuBLAS figure; the
-    # fraction of the burst figure is reported beside it
-    tens = peaks["bf16_tflops_sustained"]
-    tens_burst = peaks["bf16_tflops"]
+    # the statistics kernel runs for milliseconds at a time between the other
+    # stages, at the clocks of a short burst: its fraction is taken of the
+    # burst cuBLAS figure; the sustained (power-capped) figure is given beside it
+    tens = peaks["bf16_tflops"]
+    tens_sust = peaks["bf16_tflops_sustained"]
     kernels = {
         "mapped_av": {"bound": "hbm", "achieved": av_gbs, "peak": hbm, "unit": "GB/s",
                       "frac": av_gbs / hbm, "ms": t_av,
                       "algorithmic_bytes": alg["av_bytes"]},
         "block_stats": {"bound": "tensor", "achieved": stats_tf, "peak": tens,
                         "unit": "TFLOP/s", "frac": stats_tf / tens, "ms": t_stats,
-                        "peak_kind": "sustained bf16 (kernel timed inside a long step loop)",
-                        "frac_of_burst_peak": stats_tf / tens_burst,
+                        "peak_kind": "burst bf16",
+                        "frac_of_sustained_peak": stats_tf / tens_sust,
                         "algorithmic_flops": alg["stats_flops"]},
         "select_extract": {"bound": "hbm", "achieved": ext_gbs, "peak": hbm, "unit": "GB/s",
                            "frac": ext_gbs / hbm, "ms": t_sel,
@@ -464,7 +472,7 @@ def bench_ours(args, wl, rank, world, local_rank):
         "mapped_av_gbs": av_gbs, "mapped_av_hbm_frac": av_gbs / hbm,
         "compress_tokens_per_s": wl.ntok / ((t_stats + t_sel) * 1e-3),
         "stats_tensor_frac": stats_tf / tens,
-        "stats_tensor_frac_of_burst": stats_tf / tens_burst,
+        "stats_tensor_frac_of_sustained": stats_tf / tens_sust,
         "layer_prefill_ms": t_av,
         "dense_sdpa_ms_context": dense_ms,
         "stage_ms": {"block_stats": t_stats, "select_extract": t_sel, "mapped_av": t_av},
@@ -485,6 +493,159 @@ def bench_ours(args, wl, rank, world, local_rank):
 LAUNCHES_PER_RANGE = 12
 
 
+def bench_rounds(args):
+    """Round-level selection on the multi-turn workload (one GPU)."""
+    from cross_model_attention_block_b200 import mapflow as mfb
+    wl = synth.workloads()["multi_turn_rounds_n8192"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ctx = mfb.Context.make(wl.lengths, wl.Hs, wl.d, wl.B, wl.band_bias, wl.band_width,
+                           wl.torch_dtype, device=dev)
+    layers = [tuple(t.to(dev) for t in synth.sender_layer(wl, l) + synth.receiver_layer(wl, 0, l))
+              for l in range(wl.sender_layers)]
+    nqb, nblocks = ctx.layout_sizes()
+    lse = torch.empty((wl.Hs, wl.ntok), dtype=torch.float32, device=dev)
+    mass = torch.empty((nblocks,), dtype=torch.float32, device=dev)
+    cache = mfb.Cache(ctx, device=dev)
+    blocks = mfb.Cache(ctx, device=dev)
+    O = torch.empty((wl.ntok, wl.Hr, wl.d), dtype=wl.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    mapped = range(wl.watershed, wl.sender_layers)
+
+    def step(m=None):
+        rec = (lambda i: m[i].record(stream)) if m else (lambda i: None)
+        Qw, Kw = layers[wl.watershed][:2]
+        rec(0)
+        mfb.block_stats(ctx, Qw, Kw, lse=lse, mass=mass)
+        mfb.select_rounds(ctx, mass, wl.rounds[0], wl.tau, cache=cache)
+        rec(1)
+        for l in mapped:
+            Q, K, V, W = layers[l]
+            mfb.block_stats(ctx, Q, K, lse=lse, mass=mass)
+            mfb.extract(ctx, Q, K, lse, cache)
+            mfb.mapped_av(cache, wl.Hr, W, V, wl.Hkv, O=O, workspace=getattr(cache, "_av_ws", None))
+        rec(2)
+
+    for _ in range(args.warmup):
+        step()
+    mfb.sync_status()
+    marks = [[ev() for _ in range(3)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    for k in range(args.steps):
+        step(marks[k])
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    mfb.sync_status()
+    t = np.array([[m[0].elapsed_time(m[1]), m[1].elapsed_time(m[2])] for m in marks]).mean(0)
+    # the block selection of the watershed layer at the same tau, for the kept fraction
+    Qw, Kw = layers[wl.watershed][:2]
+    mfb.block_stats(ctx, Qw, Kw, lse=lse, mass=mass)
+    mfb.select_extract(ctx, Qw, Kw, lse, mass, wl.tau, cache=blocks)
+    mfb.sync_status()
+    ms = float(t.sum())
+    line = {
+        "mode": "rounds", "metric": "round-level selection: tokens/s of one step (selection at "
+        "the watershed layer, then statistics, extraction and the fused kernel on every later "
+        "layer)", "value": wl.ntok / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.ntok, "rounds": len(wl.rounds[0]) - 1,
+                   "sender_layers": wl.sender_layers, "watershed": wl.watershed,
+                   "mapped_layers": len(mapped), "Hs": wl.Hs, "Hr": wl.Hr, "Hkv": wl.Hkv,
+                   "B": wl.B, "tau": wl.tau},
+        "stage_ms": {"watershed_stats_and_round_selection": float(t[0]),
+                     "mapped_layers": float(t[1]),
+                     "per_mapped_layer": float(t[1]) / len(mapped)},
+        "kept_blocks": {"rounds": cache.nnz, "blocks_same_tau": blocks.nnz,
+                        "causal": nblocks},
+        "cache_gb_per_layer": {"rounds": cache.nnz * wl.Hs * wl.B * wl.B * 2 / 1e9,
+                               "blocks_same_tau": blocks.nnz * wl.Hs * wl.B * wl.B * 2 / 1e9},
+        "clocks": clk,
+        "gpu_launches": args.steps * (9 + len(mapped) * 9),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def bench_overlap(args):
+    """Receiver prefill: fetch of a mapped layer's cache from pinned host memory
+    overlapped with the recompute of the receiver's first layers (one GPU)."""
+    import torch.nn.functional as F
+    from cross_model_attention_block_b200 import mapflow as mfb
+    from cross_model_attention_block_b200 import overlap as ov
+    wl = synth.workloads()["multi_receiver_n16384"]
+    n_recompute, chunks = 2, 8
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ctx = mfb.Context.make(wl.lengths, wl.Hs, wl.d, wl.B, wl.band_bias, wl.band_width,
+                           wl.torch_dtype, device=dev)
+    Q, K = (t.to(dev) for t in synth.sender_layer(wl, 0))
+    lse, mass = mfb.block_stats(ctx, Q, K)
+    src = mfb.select_extract(ctx, Q, K, lse, mass, wl.tau)
+    mfb.sync_status()
+    nnz = src.nnz
+    host = mfb.Cache(ctx, capacity=nnz, device="cpu", pin=True)
+    mfb.cache_offload(src, host)
+    torch.cuda.synchronize()
+    del src, Q, K
+    target = mfb.Cache(ctx, capacity=nnz, device=dev)
+    V, W = (t.to(dev) for t in synth.receiver_layer(wl, 0, 0))
+    O = torch.empty((wl.ntok, wl.Hr, wl.d), dtype=wl.torch_dtype, device=dev)
+    layer = ov.MappedLayer(host, target, W, V, O)
+    g = torch.Generator(device=dev).manual_seed(11)
+    q = torch.randn(1, wl.Hr, wl.ntok, wl.d, device=dev, dtype=wl.torch_dtype, generator=g)
+    kv = torch.randn(1, wl.Hkv, wl.ntok, wl.d, device=dev, dtype=wl.torch_dtype, generator=g)
+    # stand-in for one of the receiver's own first layers (dense causal attention)
+    recompute = [lambda: F.scaled_dot_product_attention(q, kv, kv, is_causal=True,
+                                                        enable_gqa=True)] * n_recompute
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    copy = torch.cuda.Stream()
+
+    def timed(fn):
+        a, b = ev(), ev()
+        a.record(stream)
+        out = fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b), a, out
+
+    res = {"serial": [], "overlapped": [], "fetch": [], "recompute": [], "mapped": []}
+    for k in range(args.warmup + args.steps):
+        t_s, _, _ = timed(lambda: ov.prefill(recompute, [layer], wl.Hr, wl.Hkv, chunks,
+                                             serial=True))
+        t_o, a, evs = timed(lambda: ov.prefill(recompute, [layer], wl.Hr, wl.Hkv, chunks,
+                                               copy_stream=copy))
+        t_f = a.elapsed_time(evs[-1])          # start to the last range landed
+        t_r, _, _ = timed(lambda: [f() for f in recompute])
+        t_m, _, _ = timed(lambda: [mfb.mapped_av(target, wl.Hr, W, V, wl.Hkv, O=O, qb_range=r)
+                                   for r in ov.chunk_ranges(target.nqb, chunks)])
+        if k >= args.warmup:
+            for key, v in (("serial", t_s), ("overlapped", t_o), ("fetch", t_f),
+                           ("recompute", t_r), ("mapped", t_m)):
+                res[key].append(v)
+    mfb.sync_status()
+    med = {k: float(np.median(v)) for k, v in res.items()}
+    fetch_bytes = (nnz * wl.Hs * wl.B * wl.B * 2 + 4 * nnz + 16 * (target.nqb + 1))
+    line = {
+        "mode": "overlap", "metric": "receiver prefill ms: cache fetch from host memory "
+        "overlapped with the early-layer recompute, against the same calls in series",
+        "value": med["overlapped"], "unit": "ms", "higher_is_better": False, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.ntok, "recompute_layers": n_recompute,
+                   "recompute_stand_in": "torch causal SDPA (Hr query heads, Hkv KV heads)",
+                   "mapped_layers": 1, "chunks": chunks, "fetch_gb": fetch_bytes / 1e9,
+                   "source": "pinned host memory"},
+        "serial_ms": med["serial"], "overlapped_ms": med["overlapped"],
+        "saved_ms": med["serial"] - med["overlapped"],
+        "fetch_ms": med["fetch"], "fetch_gbs": fetch_bytes / (med["fetch"] * 1e-3) / 1e9,
+        "recompute_ms": med["recompute"], "mapped_ms": med["mapped"],
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -493,7 +654,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_bf16_n32768")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["path", "rounds", "overlap"], default="path")
     args = ap.parse_args(argv)
+    if args.mode != "path" and args.impl == "ours":
+        return bench_rounds(args) if args.mode == "rounds" else bench_overlap(args)
     wl = synth.workloads()[args.workload]
     rank, world, local_rank = rank_env()
     if args.impl == "reference":

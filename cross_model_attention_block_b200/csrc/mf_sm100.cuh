@@ -331,5 +331,21 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// exp2_fma on two lanes at once, on the packed f32x2 FMA pipe: the same range
+// reduction (rounding add of 1.5 * 2^23, f = x - j) and polynomial.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 j = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);
+  float2 q = ffma2(make_float2(kExp2C4, kExp2C4), f, make_float2(kExp2C3, kExp2C3));
+  q = ffma2(q, f, make_float2(kExp2C2, kExp2C2));
+  q = ffma2(q, f, make_float2(kExp2C1, kExp2C1));
+  q = ffma2(q, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
 }  // namespace sm100
 }  // namespace mf

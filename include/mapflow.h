@@ -323,15 +323,15 @@ mf_status mf_cache_fetch(const mf_csr_cache* host_src, mf_csr_cache* dev_dst, in
                          int64_t qb_end, mf_stream_t stream);
 
 /* Diagnostic, not on the hot path: y[i] = 2^x[i] by the FMA-pipe
- * exponential written for the block-statistics epilogue (x = j + f,
- * j = round(x); 2^f from a degree-4 polynomial with relative minimax error
- * 2.7e-6 on [-1/2, 1/2]; 2^j added to the exponent).  Measured slower there
- * than the MUFU exponential, so the statistics kernel currently computes none
- * of its exponentials with it.  Meant for x <= 0; x below -125 is clamped to
- * -125.  x, y: device float arrays of n elements (they may be the same
- * array).  Lets tests hold it against CUDA's exp2f.  Errors:
- * MF_ERR_INVALID_ARG (n < 0, or a NULL array with n > 0), MF_ERR_CUDA (launch
- * failure). */
+ * exponential of the block-statistics kernel, which computes 2 of every 8 of
+ * its exponentials this way (the rest on MUFU): x = j + f, j = round(x); 2^f
+ * from a degree-4 polynomial with relative minimax error 2.7e-6 on
+ * [-1/2, 1/2]; 2^j added to the exponent; two lanes per packed f32x2
+ * instruction (pairs of elements; a last odd element by the scalar form).
+ * Meant for x <= 0; x below -125 is clamped to -125.  x, y: device float
+ * arrays of n elements (they may be the same array).  Lets tests hold it
+ * against CUDA's exp2f.  Errors: MF_ERR_INVALID_ARG (n < 0, or a NULL array
+ * with n > 0), MF_ERR_CUDA (launch failure). */
 mf_status mf_exp2_fma_eval(const float* x, float* y, int64_t n, mf_stream_t stream);
 
 /* Which kernels the calls above run for a shape (host only; nothing is

@@ -322,54 +322,124 @@ def rank_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def layer_jobs(wl, rank, world):
+    """The layers this rank runs: (sender layers [index], receiver layers
+    [(receiver, layer, sender index)]).  One-layer workloads: sender 0 and
+    its receiver; the multi-receiver workload: every sender layer and every
+    receiver layer through the layer table at N = 1, whole sender layers with
+    the receiver layers that read them at N > 1."""
+    if wl.sender_layers == 1:
+        return [0], [(0, 0, 0)]
+    if world == 1:
+        senders = list(range(wl.sender_layers))
+        readers = [(r, l) for r, (_, n, _) in enumerate(wl.receivers) for l in range(n)]
+    else:
+        senders, readers = partition.layer_split(wl.sender_layers, wl.receivers, world, rank)
+    return senders, [(r, l, wl.receivers[r][2][l]) for r, l in readers]
+
+
+def layer_inputs(wl, senders, receivers):
+    """Host tensors: {sender layer: (Q, K)}, {(receiver, layer): (V, W)}."""
+    if wl.sender_layers == 1:
+        x = synth.single_layer(wl)
+        return {0: (x.Q, x.K)}, {(0, 0): (x.V, x.W)}
+    return ({s: synth.sender_layer(wl, s) for s in senders},
+            {(r, l): synth.receiver_layer(wl, r, l) for r, l, _ in receivers})
+
+
 def bench_ours(args, wl, rank, world, local_rank):
     from cross_model_attention_block_b200 import mapflow as mfb
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    x = synth.single_layer(wl)
     ctx = mfb.Context.make(wl.lengths, wl.Hs, wl.d, wl.B, wl.band_bias, wl.band_width,
                            wl.torch_dtype, device=dev)
-    Q, K, V, W = (t.to(dev) for t in (x.Q, x.K, x.V, x.W))
     nqb, nblocks = ctx.layout_sizes()
-    plan = rank_plan(wl, rank, world)
+    senders, receivers = layer_jobs(wl, rank, world)
+    host_s, host_r = layer_inputs(wl, senders, receivers)
+    # query-block ranges of a sender layer on this rank: the rank's share of a
+    # one-layer workload, the whole layer when layers are split
+    plan = rank_plan(wl, rank, world) if wl.sender_layers == 1 else [(0, nqb)]
+    # V in its page pool where the workload says so (16-token pages, a random
+    # permutation of the pages of the whole batch)
+    host_pages = {}
+    contig_v = {key: V for key, (V, W) in host_r.items()}  # the oracle's V
+    if wl.paged:
+        for key, (V, W) in host_r.items():
+            pool, table = synth.paged_v(V, wl.lengths, synth.page_rng(wl))
+            host_r[key] = (pool, W)
+            host_pages[key] = table
+    # per step, the inputs: Q, K of every sender layer, V (or its pool) and W
+    # of every receiver layer, and the page tables
+    in_keys = ([("Q", s) for s in senders] + [("K", s) for s in senders]
+               + [("V", k) for k in host_r] + [("W", k) for k in host_r]
+               + [("T", k) for k in host_pages])
+    host_in = {}
+    for s in senders:
+        host_in[("Q", s)], host_in[("K", s)] = host_s[s]
+    for k, (V, W) in host_r.items():
+        host_in[("V", k)], host_in[("W", k)] = V, W
+    for k, t in host_pages.items():
+        host_in[("T", k)] = t
+    dev_in = {k: host_in[k].to(dev) for k in in_keys}
     lse = torch.empty((wl.Hs, wl.ntok), dtype=torch.float32, device=dev)
     mass = torch.empty((nblocks,), dtype=torch.float32, device=dev)
-    # one cache per range, sized to the range's causal blocks
-    caches = [mfb.Cache(ctx, capacity=ctx.range_blocks(a, b), device=dev) for a, b in plan]
-    O = torch.empty((wl.ntok, wl.Hr, wl.d), dtype=wl.torch_dtype, device=dev)
+    # one cache per (sender layer, range), sized to the range's causal blocks
+    caches = {(s, r): mfb.Cache(ctx, capacity=ctx.range_blocks(*r), device=dev)
+              for s in senders for r in plan}
+    outs = {(r, l): torch.empty((wl.ntok, wl.Hr, wl.d), dtype=wl.torch_dtype, device=dev)
+            for r, l, _ in receivers}
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
-    def run(Qd, Kd, Vd, Wd, Od, marks=None):
-        # stage by stage over this rank's ranges: statistics, then selection
-        # and extraction, then the fused kernel
-        if marks is not None:
-            marks[0].record(stream)
-        for r in plan:
-            mfb.block_stats(ctx, Qd, Kd, lse=lse, mass=mass, qb_range=r)
-        if marks is not None:
-            marks[1].record(stream)
-        for r, c in zip(plan, caches):
-            mfb.select_extract(ctx, Qd, Kd, lse, mass, wl.tau, cache=c, qb_range=r)
-        if marks is not None:
-            marks[2].record(stream)
-        for r, c in zip(plan, caches):
-            mfb.mapped_av(c, wl.Hr, Wd, Vd, wl.Hkv, O=Od, workspace=getattr(c, "_av_ws", None),
-                          qb_range=r)
-        if marks is not None:
-            marks[3].record(stream)
+    def run(din, dout, marks=None):
+        """One step: every sender layer's statistics, then its selection and
+        extraction (range by range), then every receiver layer's fused
+        kernel on its sender layer's cache.  marks: list collecting
+        (stage, start event, end event)."""
+        def timed(stage, fn):
+            if marks is None:
+                fn()
+                return
+            a, b = ev(), ev()
+            a.record(stream)
+            fn()
+            b.record(stream)
+            marks.append((stage, a, b))
+
+        for s in senders:
+            Qd, Kd = din[("Q", s)], din[("K", s)]
+            timed(0, lambda: [mfb.block_stats(ctx, Qd, Kd, lse=lse, mass=mass, qb_range=r)
+                              for r in plan])
+            timed(1, lambda: [mfb.select_extract(ctx, Qd, Kd, lse, mass, wl.tau,
+                                                 cache=caches[(s, r)], qb_range=r)
+                              for r in plan])
+        for rr, l, s in receivers:
+            key = (rr, l)
+            table = din.get(("T", key))
+
+            def av():
+                for r in plan:
+                    c = caches[(s, r)]
+                    mfb.mapped_av(c, wl.Hr, din[("W", key)], din[("V", key)], wl.Hkv,
+                                  page_table=table, O=dout[key],
+                                  workspace=getattr(c, "_av_ws", None), qb_range=r)
+            timed(2, av)
 
     def step(marks=None):
-        run(Q, K, V, W, O, marks)
+        run(dev_in, outs, marks)
 
     for _ in range(args.warmup):
         step()
     mfb.sync_status()
-    nnz = sum(c.nnz for c in caches)
-    alg = algorithmic(wl, nnz, plan)
+    nnz = {s: sum(caches[(s, r)].nnz for r in plan) for s in senders}
+    alg_s = [algorithmic(wl, nnz[s], plan) for s in senders]
+    alg = {"stats_flops": sum(a["stats_flops"] for a in alg_s),
+           "extract_bytes": sum(a["extract_bytes"] for a in alg_s),
+           "av_bytes": sum(algorithmic(wl, nnz[s], plan)["av_bytes"] for _, _, s in receivers),
+           "map_bytes": sum(a["map_bytes"] for a in alg_s)}
 
-    marks = [[ev() for _ in range(4)] for _ in range(args.steps)]
+    marks = [[] for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -385,36 +455,38 @@ def bench_ours(args, wl, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     ms = t_start.elapsed_time(t_end)
-    stage = np.array([[m[i].elapsed_time(m[i + 1]) for i in range(3)] for m in marks])
+    stage = np.zeros((args.steps, 3))
+    for k, m in enumerate(marks):
+        for st, a, b in m:
+            stage[k, st] += a.elapsed_time(b)
     stage_ms = stage.mean(axis=0)
     ms = max_over_ranks(ms, world, dev)
     mfb.sync_status()
 
     # context only: dense causal GQA attention of the same receiver layer
     # (torch scaled_dot_product_attention, bf16, per sequence), the cost the
-    # fused kernel stands in for
+    # fused kernel stands in for (per receiver layer)
     dense_ms = dense_attention_ms(wl, dev, stream, ev, args.warmup, min(args.steps, 10))
     dense_ms = max_over_ranks(dense_ms, world, dev)
 
     # end to end through the C ABI: every step copies its inputs in from
-    # pinned host memory and its output back, as a serving loop would: the
+    # pinned host memory and its outputs back, as a serving loop would: the
     # copies run on two copy streams into double-buffered device tensors, so
     # step k's H2D and step k-1's D2H overlap step k-1's and k's kernels
-    pin = lambda t: t.pin_memory()  # noqa: E731
-    hQ, hK, hV, hW = pin(x.Q), pin(x.K), pin(x.V), pin(x.W)
-    hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
-    dIn = [tuple(torch.empty_like(t, device=dev) for t in (hQ, hK, hV, hW)) for _ in range(2)]
-    dO = [O, torch.empty_like(O)]
+    hIn = {k: host_in[k].pin_memory() for k in in_keys}
+    hOut = {k: torch.empty(o.shape, dtype=o.dtype).pin_memory() for k, o in outs.items()}
+    dIn = [dev_in, {k: torch.empty_like(t) for k, t in dev_in.items()}]
+    dOut = [outs, {k: torch.empty_like(o) for k, o in outs.items()}]
     h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     in_ready = [ev() for _ in range(2)]
     used = [ev() for _ in range(2)]      # step's kernels done with buffer set b
-    out_read = [ev() for _ in range(2)]  # output b copied back
+    out_read = [ev() for _ in range(2)]  # outputs b copied back
 
     def e2e_run(nsteps):
         def h2d(b):
             with torch.cuda.stream(h2d_s):
-                for d, h in zip(dIn[b], (hQ, hK, hV, hW)):
-                    d.copy_(h, non_blocking=True)
+                for k in in_keys:
+                    dIn[b][k].copy_(hIn[k], non_blocking=True)
                 in_ready[b].record(h2d_s)
 
         h2d_s.wait_stream(stream)  # nothing starts before the timed region does
@@ -427,12 +499,13 @@ def bench_ours(args, wl, rank, world, local_rank):
                 h2d(1 - b)
             stream.wait_event(in_ready[b])
             if k >= 2:
-                stream.wait_event(out_read[b])     # step k-2's output has been read back
-            run(*dIn[b], dO[b])
+                stream.wait_event(out_read[b])     # step k-2's outputs have been read back
+            run(dIn[b], dOut[b])
             used[b].record(stream)
             d2h_s.wait_event(used[b])
             with torch.cuda.stream(d2h_s):
-                hO.copy_(dO[b], non_blocking=True)
+                for key, o in dOut[b].items():
+                    hOut[key].copy_(o, non_blocking=True)
                 out_read[b].record(d2h_s)
         stream.wait_stream(d2h_s)
 
@@ -445,14 +518,18 @@ def bench_ours(args, wl, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     mfb.sync_status()
-    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hW))
-    d2h = hO.numel() * hO.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in hIn.values())
+    d2h = sum(t.numel() * t.element_size() for t in hOut.values())
+    # the CPU baseline's inputs: the first sender layer and its first reader
+    s0 = senders[0]
+    k0 = next((rr, l) for rr, l, s in receivers if s == s0)
+    x = synth.LayerInputs(*host_s[s0], contig_v[k0], host_r[k0][1])
 
     if rank != 0:
         return
     peaks, src = load_peaks()
     ms_step = ms / args.steps
-    tokens = wl.ntok  # one layer, split across the ranks
+    tokens = wl.ntok  # the context of one step, split across the ranks
     t_stats, t_sel, t_av = stage_ms
     av_gbs = alg["av_bytes"] / (t_av * 1e-3) / 1e9
     stats_tf = alg["stats_flops"] / (t_stats * 1e-3) / 1e12
@@ -489,33 +566,41 @@ def bench_ours(args, wl, rank, world, local_rank):
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "tokens": wl.ntok, "Hs": wl.Hs, "Hr": wl.Hr,
                    "Hkv": wl.Hkv, "d": wl.d, "B": wl.B, "tau": wl.tau,
-                   "kept_blocks": nnz, "causal_blocks": nblocks,
+                   "sender_layers": len(senders), "receiver_layers": len(receivers),
+                   "paged_v": bool(wl.paged),
+                   "kept_blocks": sum(nnz.values()), "causal_blocks": nblocks * len(senders),
                    "map_gb": alg["map_bytes"] / 1e9,
                    "l2": "inputs larger than L2 (kept map >> 126 MB); no flush",
-                   "parallelism": (f"query-block ranges x{world} (rank 0: {plan})"
-                                   if world > 1 else "single GPU")},
+                   "parallelism": ("single GPU" if world == 1 else
+                                   f"query-block ranges x{world} (rank 0: {plan})"
+                                   if wl.sender_layers == 1 else
+                                   f"sender layers with their readers x{world} "
+                                   f"(rank 0: {senders})")},
         "mapped_av_gbs": av_gbs, "mapped_av_hbm_frac": av_gbs / hbm,
-        "compress_tokens_per_s": wl.ntok / ((t_stats + t_sel) * 1e-3),
+        "compress_tokens_per_s": wl.ntok * len(senders) / ((t_stats + t_sel) * 1e-3),
         "stats_tensor_frac": stats_tf / tens,
         "stats_tensor_frac_of_sustained": stats_tf / tens_sust,
-        "layer_prefill_ms": t_av,
+        "layer_prefill_ms": t_av / len(receivers),
         "dense_sdpa_ms_context": dense_ms,
         "stage_ms": {"block_stats": t_stats, "select_extract": t_sel, "mapped_av": t_av},
         "roofline": roof, "kernels": kernels,
         "clocks": clk,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * LAUNCHES_PER_RANGE * len(plan),
+        "gpu_launches": args.steps * len(plan) * (LAUNCHES_COMPRESS * len(senders)
+                                                  + LAUNCHES_MAPPED * len(receivers)),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_sample(wl, x)
     print(json.dumps(line), flush=True)
 
 
-# kernels of ours launched per query-block range and step: stats (meta, stats,
-# mass reduce), select and extract (meta, qb map, select, scan, fill,
-# extract), mapped AV (group meta, V regrouping, fused kernel)
-LAUNCHES_PER_RANGE = 12
+# kernels of ours launched per query-block range and step: per sender layer,
+# stats (meta, stats, mass reduce) and select and extract (meta, qb map,
+# select, scan, fill, extract); per receiver layer, mapped AV (group meta, V
+# regrouping, fused kernel)
+LAUNCHES_COMPRESS = 9
+LAUNCHES_MAPPED = 3
 
 
 def bench_rounds(args):

@@ -88,3 +88,30 @@ def test_bench_rank_plans_cover_the_layer_once():
             units = [bench.plan_units(wl, p) for p in plans]
             assert sum(u[0] for u in units) == full_rows
             assert sum(u[1] for u in units) == full_pairs
+
+
+def test_bench_layer_jobs():
+    """bench.py's layers per rank: one-layer workloads run sender 0 and its
+    receiver; the multi-receiver workload runs all 8 sender layers and all
+    6 + 4 receiver layers at N = 1, and at N > 1 the ranks' sender layers
+    cover the 8 once, each receiver layer on the rank of its sender layer."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from cross_model_attention_block_b200 import synth
+    w2 = synth.workloads()["large_bf16_n32768"]
+    assert bench.layer_jobs(w2, 0, 1) == ([0], [(0, 0, 0)])
+    assert bench.layer_jobs(w2, 1, 4) == ([0], [(0, 0, 0)])
+    w3 = synth.workloads()["multi_receiver_n16384"]
+    s, r = bench.layer_jobs(w3, 0, 1)
+    assert s == list(range(8)) and len(r) == 10
+    assert all(w3.receivers[rr][2][l] == src for rr, l, src in r)
+    for world in (2, 4, 8):
+        all_s, all_r = [], []
+        for rank in range(world):
+            s, r = bench.layer_jobs(w3, rank, world)
+            assert all(src in s for _, _, src in r)
+            all_s += s
+            all_r += [(rr, l) for rr, l, _ in r]
+        assert sorted(all_s) == list(range(8))
+        assert sorted(all_r) == sorted((rr, l) for rr, (_, n, _) in enumerate(w3.receivers)
+                                       for l in range(n))

@@ -46,7 +46,7 @@ typedef struct CUstream_st* mf_stream_t; /* same object as cudaStream_t */
 typedef enum {
   MF_OK = 0,
   MF_ERR_INVALID_ARG = 1,  /* null pointer, inconsistent sizes */
-  MF_ERR_UNSUPPORTED = 2,  /* a shape this build has no kernel for */
+  MF_ERR_UNSUPPORTED = 2,  /* a shape the library has no kernel for */
   MF_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
   MF_ERR_CUDA = 4,         /* a CUDA runtime call or a launch failed */
   MF_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up */

@@ -51,6 +51,7 @@ struct Params {
   const int32_t* cu_qb;    // [nseq+1]
   int ntiles;
   int Hs;
+  int head_group;  // extraction: heads per CTA group (head innermost)
   int B;
   int band_width;
   float scale2;            // log2(e) / sqrt(d)
@@ -87,21 +88,6 @@ __device__ __forceinline__ float transpose_reduce32(float* v, int lane) {
     }
   }
   return v[0];
-}
-
-// AND of a predicate over one of the four epilogue warpgroups (named
-// barriers 6..9).
-__device__ __forceinline__ bool group_all(int wg, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(uint32_t(v)), "r"(6 + wg)
-      : "memory");
-  return r != 0;
 }
 
 // ------------------------------------------------- statistics, four groups
@@ -393,11 +379,19 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 //
 // Extraction with four epilogue warpgroups: as in k_stats_wide, the two
 // groups of a tile parity (counted over the kept tiles only) split the
-// tile's columns, so each group extracts one
-// 64-key chunk per tile into its own 16 KB staging buffer and stores it with
-// TMA right away (B = 128: half the block's lines; B = 64: the chunk's key
-// block in each of the two row blocks).  A group waits for its previous
-// stores to finish reading its buffer before writing it again.
+// tile's columns, so each group extracts one 64-key chunk per tile into its
+// own 16 KB staging buffer.  A warp's 32 rows fill 8 consecutive 128-byte
+// lines of every 16-key group there, so each warp stores its own lines with
+// TMA (four 8-line boxes per tile) and waits only for its own previous
+// stores: no barrier inside the group.  The staging tile is laid out in the
+// stores' 128-byte swizzle (16-byte chunk ^ line % 8), which spreads the 8
+// lanes of a shared-memory store phase over all 32 banks; the layout in the
+// cache is unchanged.  CTAs take heads in groups of kHeadGroup, the head
+// innermost, so the heads' 128-byte pieces of a cache line (adjacent in the
+// cache layout) are written at about the same time, while the group's K
+// stays in L2.
+constexpr int kHeadGroup = 8;
+
 struct SmemWideX {
   uint8_t q[kTileBytes];
   uint8_t k[3][kTileBytes];
@@ -412,11 +406,6 @@ struct SmemWideX {
   uint32_t tmem_base;
 };
 
-// One epilogue warpgroup of the four (named barriers 6..9).
-__device__ __forceinline__ void group4_sync(int eg) {
-  asm volatile("bar.sync %0, 128;" ::"r"(6 + eg) : "memory");
-}
-
 template <int BB>
 __global__ void __launch_bounds__(kWideThreads, 1)
     k_extract_wide(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -426,8 +415,14 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   SmemWideX& sm = *reinterpret_cast<SmemWideX*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x / p.ntiles;
-  const int w = blockIdx.x % p.ntiles;
+  // heads in groups of head_group, the head innermost: the CTAs writing
+  // neighbouring 128-byte pieces of a cache line run at about the same time
+  const int per = p.ntiles * p.head_group;
+  const int hg = blockIdx.x / per;
+  const int gsz = min(p.head_group, p.Hs - hg * p.head_group);
+  const int rem = blockIdx.x - hg * per;
+  const int h = hg * p.head_group + rem % gsz;
+  const int w = rem / gsz;
   const int s = p.tiles[2 * w], t = p.tiles[2 * w + 1];
   const int seq0 = p.cu_seqlens[s];
   const int L = p.cu_seqlens[s + 1] - seq0;
@@ -523,21 +518,22 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const bool valid = ri < L;
     const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
     const int W = p.band_width;
-    const bool leader = (threadIdx.x & 127) == 0;
     const float lse2 = valid ? p.lse[int64_t(h) * p.ntok + seq0 + ri] * kLog2e : 0.f;
     const int rb = r & (BB - 1);                          // row within the block
     const int lrow = ((rb >> 3) << 1) + ((rb & 7) >> 2);  // line of this row, key group 0
     const int cbase = (rb & 3) << 1;                       // chunk of keys 0-7
-    uint8_t* buf = sm.out[eg];
+    // The warp's 32 rows fill 8 consecutive lines of every 16-key group of its
+    // (row block's) staging area: it writes and stores them on its own.
+    const int a = (BB == 128) ? 0 : (quarter >> 1);               // row block (B = 64)
+    const int wl = (BB == 128) ? 8 * quarter : 8 * (quarter & 1);  // first line per key group
+    uint8_t* sub = sm.out[eg] + a * 8192;
     int n = 0;
     for (int kt = 0; kt <= t; ++kt) {
       if (!tile_needed<BB>(sm.slots, kt)) continue;
       if ((n & 1) != par) { ++n; continue; }
       const int sb = par;
-      bool got = mbar_wait(&sm.s_full[sb], (n >> 1) & 1, p.status);
-      // the group meets at named barriers below: it leaves the loop together
-      got = group_all(eg, got);
-      if (!got) break;
+      const bool got = mbar_wait(&sm.s_full[sb], (n >> 1) & 1, p.status);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       float v[64];
       tmem_ld32(lane_addr + sb * 128 + hc * 64, v);
@@ -560,12 +556,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         }
       }
       const int kb = (BB == 128) ? kt : 2 * kt + hc;
-      const bool kept = sm.slots[(BB == 128) ? 0 : (r >> 6)][kb] >= 0;
-      // the group's previous stores are done reading the staging buffer
-      if (leader) bulk_wait_read<0>();
-      group4_sync(eg);
-      if (kept) {
-        uint8_t* sub = buf + ((BB == 128) ? 0 : (r >> 6) * 8192);
+      const int e = sm.slots[a][kb];
+      if (e >= 0) {
+        // the warp's previous stores are done reading its lines
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
 #pragma unroll
         for (int kgl = 0; kgl < 4; ++kgl) {
           uint8_t* line = sub + (kgl * (BB / 4) + lrow) * 128;
@@ -581,29 +576,25 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                   __floats2bfloat162_rn(valid ? ex2(x.x) : 0.f, valid ? ex2(x.y) : 0.f);
               w4[k] = *reinterpret_cast<uint32_t*>(&pr);
             }
-            *reinterpret_cast<uint4*>(line + (((cbase | c) ^ (h & 7)) << 4)) =
+            *reinterpret_cast<uint4*>(line + ((((cbase | c) ^ (h & 7)) ^ (lrow & 7)) << 4)) =
                 make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
-      }
-      fence_proxy_async_smem();
-      group4_sync(eg);
-      if (leader) {
-        if (BB == 128) {
-          const int e = sm.slots[0][kt];
-          if (e >= 0) tma_store_4d(&tmV, buf, 0, h, hc * 128, int32_t(e));
-        } else {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int l0 = (BB == 128) ? hc * 128 : 0;
 #pragma unroll
-          for (int a = 0; a < 2; ++a) {
-            const int e = sm.slots[a][kb];
-            if (e >= 0) tma_store_4d(&tmV, buf + a * 8192, 0, h, 0, int32_t(e));
+          for (int kgl = 0; kgl < 4; ++kgl) {
+            const int ln = kgl * (BB / 4) + wl;
+            tma_store_4d(&tmV, sub + ln * 128, 0, h, l0 + ln, int32_t(e));
           }
+          bulk_commit();
         }
-        bulk_commit();
       }
       ++n;
     }
-    if (leader) bulk_wait_all<0>();
+    if (lane == 0) bulk_wait_all<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -753,13 +744,13 @@ cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const QbRa
   if (e != cudaSuccess) return e;
   e = make_tmap_2d_bf16(&tk, K, uint64_t(sz.ntok), cols, 64, qk::kTile, true);
   if (e != cudaSuccess) return e;
-  // one store writes one 64-key chunk of an (entry, head): B = 128, half the
-  // block's lines; B = 64, all of them
+  // one store writes 8 lines of an (entry, head): one warp's rows of one
+  // 16-key group, from a staging tile in the 128-byte swizzle
   const uint64_t nl = uint64_t(d.B) * uint64_t(d.B) / 64;
   const uint64_t dims[4] = {64, uint64_t(d.Hs), nl, uint64_t(capacity)};
   const uint64_t strides[3] = {128, uint64_t(d.Hs) * 128, nl * uint64_t(d.Hs) * 128};
-  const uint32_t box[4] = {64, 1, uint32_t(nl < 128 ? nl : 128), 1};
-  e = make_tmap_bf16(&tv, values, 4, dims, strides, box, 0);
+  const uint32_t box[4] = {64, 1, 8, 1};
+  e = make_tmap_bf16(&tv, values, 4, dims, strides, box, 128);
   if (e != cudaSuccess) return e;
   qk::Params p{};
   p.cu_seqlens = d.cu_seqlens;
@@ -768,6 +759,7 @@ cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const QbRa
   p.cu_qb = m.cu_qb;
   p.ntiles = int(r.ntiles);
   p.Hs = d.Hs;
+  p.head_group = std::min(d.Hs, qk::kHeadGroup);
   p.B = d.B;
   p.band_width = d.band_width;
   p.scale2 = qk::kLog2e / sqrtf(float(d.d));

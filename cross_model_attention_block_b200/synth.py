@@ -77,7 +77,7 @@ def _varlen_lengths(n: int, lo: int, hi: int, seed: int):
 
 
 def workloads() -> dict:
-    """The five synthetic workloads, keyed by a descriptive name."""
+    """The synthetic workloads, keyed by a descriptive name."""
     w = {}
     w["tiny_f32_n512"] = Workload(
         "tiny_f32_n512", [512], Hs=4, Hr=2, Hkv=2, d=64, B=64, tau=0.9,
@@ -87,6 +87,11 @@ def workloads() -> dict:
         band_bias=2.0, band_width=256, dtype="bf16", seed=0)
     w["large_bf16_n32768"] = Workload(
         "large_bf16_n32768", [32768], Hs=40, Hr=32, Hkv=8, d=128, B=128,
+        tau=0.95, band_bias=2.0, band_width=256, dtype="bf16", seed=0)
+    # the 32K workload's shape (heads, B = 128) at 8,192 tokens: small enough for
+    # counter captures of the B = 128 kernels (a few GB on the device)
+    w["large_shape_bf16_n8192"] = Workload(
+        "large_shape_bf16_n8192", [8192], Hs=40, Hr=32, Hkv=8, d=128, B=128,
         tau=0.95, band_bias=2.0, band_width=256, dtype="bf16", seed=0)
     # one sender state (8 layers) consumed by two receivers; receiver layer l
     # of an L-layer receiver reads sender layer floor(l * 8 / L)

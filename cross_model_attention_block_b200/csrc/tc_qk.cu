@@ -386,11 +386,14 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 // stores: no barrier inside the group.  The staging tile is laid out in the
 // stores' 128-byte swizzle (16-byte chunk ^ line % 8), which spreads the 8
 // lanes of a shared-memory store phase over all 32 banks; the layout in the
-// cache is unchanged.  CTAs take heads in groups of kHeadGroup, the head
-// innermost, so the heads' 128-byte pieces of a cache line (adjacent in the
-// cache layout) are written at about the same time, while the group's K
-// stays in L2.
+// cache is unchanged.  CTAs take heads in groups of up to kHeadGroup, the
+// head innermost, so the heads' 128-byte pieces of a cache line (adjacent in
+// the cache layout) are written at about the same time; the group is cut so
+// that its K (every sequence's keys of those heads) fits kHeadGroupL2 bytes
+// and stays in L2 while the tiles run (one head when a single head's K does
+// not fit, the order of one head after another).
 constexpr int kHeadGroup = 8;
+constexpr double kHeadGroupL2 = 72.0 * 1024 * 1024;
 
 struct SmemWideX {
   uint8_t q[kTileBytes];
@@ -759,7 +762,11 @@ cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const QbRa
   p.cu_qb = m.cu_qb;
   p.ntiles = int(r.ntiles);
   p.Hs = d.Hs;
-  p.head_group = std::min(d.Hs, qk::kHeadGroup);
+  {
+    const double k_head = double(sz.ntok) * double(d.d) * 2.0;  // K bytes of one head
+    const int fit = int(std::min(double(qk::kHeadGroup), qk::kHeadGroupL2 / k_head));
+    p.head_group = std::max(1, std::min(d.Hs, fit));
+  }
   p.B = d.B;
   p.band_width = d.band_width;
   p.scale2 = qk::kLog2e / sqrtf(float(d.d));

@@ -37,8 +37,12 @@ def _small(lengths, Hs, Hr, Hkv, d, B, tau, dtype="bf16", band_bias=2.0, band_wi
     dict(lengths=[333, 65], Hs=4, Hr=4, Hkv=4, d=64, B=64, tau=0.9),
     dict(lengths=[200, 77], Hs=3, Hr=6, Hkv=3, d=128, B=128, tau=0.9, dtype="f32"),
     dict(lengths=[100, 0, 70], Hs=5, Hr=4, Hkv=2, d=64, B=64, tau=0.8, dtype="f32"),
+    # 12 sender heads: tensor-core statistics and extraction with a partial
+    # last head group (8 + 4); the fused step runs the scalar kernel
+    dict(lengths=[700, 257], Hs=12, Hr=8, Hkv=4, d=128, B=128, tau=0.95),
+    dict(lengths=[450, 1], Hs=12, Hr=8, Hkv=4, d=128, B=64, tau=0.9),
 ], ids=["bf16_b64_varlen", "bf16_b128_hs40", "bf16_b64_hs32", "bf16_d64",
-        "f32_d128_b128", "f32_empty_seq"])
+        "f32_d128_b128", "f32_empty_seq", "bf16_b128_hs12", "bf16_b64_hs12"])
 def test_small_cases_every_block(case):
     w, x, ctx, gpu = _small(**case)
     dt = w.torch_dtype

@@ -530,6 +530,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const int a = (BB == 128) ? 0 : (quarter >> 1);               // row block (B = 64)
     const int wl = (BB == 128) ? 8 * quarter : 8 * (quarter & 1);  // first line per key group
     uint8_t* sub = sm.out[eg] + a * 8192;
+    // the kept map (tens of GB) is written once: its lines leave L2 first, so
+    // the K tiles that later query tiles re-read stay
+    const uint64_t keep_out = l2_evict_first();
     int n = 0;
     for (int kt = 0; kt <= t; ++kt) {
       if (!tile_needed<BB>(sm.slots, kt)) continue;
@@ -590,7 +593,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
           for (int kgl = 0; kgl < 4; ++kgl) {
             const int ln = kgl * (BB / 4) + wl;
-            tma_store_4d(&tmV, sub + ln * 128, 0, h, l0 + ln, int32_t(e));
+            tma_store_4d_hint(&tmV, sub + ln * 128, 0, h, l0 + ln, int32_t(e), keep_out);
           }
           bulk_commit();
         }

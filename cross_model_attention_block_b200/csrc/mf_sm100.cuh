@@ -107,24 +107,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
-// Shared -> global tensor store (bulk-group completion).
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, const void* src, int32_t c0,
-                                             int32_t c1, int32_t c2, int32_t c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(m)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-
-// The same store with an L2 eviction policy (see l2_evict_first).
-__device__ __forceinline__ void tma_store_4d_hint(const CUtensorMap* m, const void* src, int32_t c0,
-                                                  int32_t c1, int32_t c2, int32_t c3,
+// Shared -> global tensor store (bulk-group completion), rank 5, with an L2
+// eviction policy (see l2_evict_first).
+__device__ __forceinline__ void tma_store_5d_hint(const CUtensorMap* m, const void* src, int32_t c0,
+                                                  int32_t c1, int32_t c2, int32_t c3, int32_t c4,
                                                   uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group.L2::cache_hint"
-      " [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(reinterpret_cast<uint64_t>(m)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+      "cp.async.bulk.tensor.5d.global.shared::cta.bulk_group.L2::cache_hint"
+      " [%0, {%2, %3, %4, %5, %6}], [%1], %7;" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "l"(policy)
       : "memory");
 }
 

@@ -380,13 +380,13 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 // Extraction with four epilogue warpgroups: as in k_stats_wide, the two
 // groups of a tile parity (counted over the kept tiles only) split the
 // tile's columns, so each group extracts one 64-key chunk per tile into its
-// own 16 KB staging buffer.  A warp's 32 rows fill 8 consecutive 128-byte
-// lines of every 16-key group there, so each warp stores its own lines with
-// TMA (four 8-line boxes per tile) and waits only for its own previous
-// stores: no barrier inside the group.  The staging tile is laid out in the
-// stores' 128-byte swizzle (16-byte chunk ^ line % 8), which spreads the 8
-// lanes of a shared-memory store phase over all 32 banks; the layout in the
-// cache is unchanged.  CTAs take heads in groups of up to kHeadGroup, the
+// own 16 KB staging buffer.  A warp's 32 rows make 8 consecutive 128-byte
+// lines of every 16-key group in the cache; the warp stages its 4 x 8 lines
+// as one 4 KB run, stores them with one TMA store per tile and waits only for
+// its own previous store: no barrier inside the group.  The run is laid out
+// in the store's 128-byte swizzle (16-byte chunk ^ line % 8), which spreads
+// the 8 lanes of a shared-memory store phase over all 32 banks; the layout in
+// the cache is unchanged.  CTAs take heads in groups of up to kHeadGroup, the
 // head innermost, so the heads' 128-byte pieces of a cache line (adjacent in
 // the cache layout) are written at about the same time; the group is cut so
 // that its K (every sequence's keys of those heads) fits kHeadGroupL2 bytes
@@ -529,7 +529,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     // (row block's) staging area: it writes and stores them on its own.
     const int a = (BB == 128) ? 0 : (quarter >> 1);               // row block (B = 64)
     const int wl = (BB == 128) ? 8 * quarter : 8 * (quarter & 1);  // first line per key group
-    uint8_t* sub = sm.out[eg] + a * 8192;
+    uint8_t* stage = sm.out[eg] + quarter * 4096;  // the warp's 4 key groups x 8 lines
     // the kept map (tens of GB) is written once: its lines leave L2 first, so
     // the K tiles that later query tiles re-read stay
     const uint64_t keep_out = l2_evict_first();
@@ -569,7 +569,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         __syncwarp();
 #pragma unroll
         for (int kgl = 0; kgl < 4; ++kgl) {
-          uint8_t* line = sub + (kgl * (BB / 4) + lrow) * 128;
+          uint8_t* line = stage + (kgl * 8 + (lrow & 7)) * 128;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t w4[4];
@@ -589,12 +589,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          const int l0 = (BB == 128) ? hc * 128 : 0;
-#pragma unroll
-          for (int kgl = 0; kgl < 4; ++kgl) {
-            const int ln = kgl * (BB / 4) + wl;
-            tma_store_4d_hint(&tmV, sub + ln * 128, 0, h, l0 + ln, int32_t(e), keep_out);
-          }
+          tma_store_5d_hint(&tmV, stage, 0, h, wl, (BB == 128) ? hc * 4 : 0, int32_t(e),
+                            keep_out);
           bulk_commit();
         }
       }
@@ -750,13 +746,16 @@ cudaError_t launch_extract_tc(const mf_attn_desc& d, const Sizes& sz, const QbRa
   if (e != cudaSuccess) return e;
   e = make_tmap_2d_bf16(&tk, K, uint64_t(sz.ntok), cols, 64, qk::kTile, true);
   if (e != cudaSuccess) return e;
-  // one store writes 8 lines of an (entry, head): one warp's rows of one
-  // 16-key group, from a staging tile in the 128-byte swizzle
+  // one store writes one warp's rows of an (entry, head): 8 lines of each of
+  // the 4 key groups of a 64-key chunk, from a staging run in the 128-byte
+  // swizzle; the lines are split as (line in its key group, key group)
   const uint64_t nl = uint64_t(d.B) * uint64_t(d.B) / 64;
-  const uint64_t dims[4] = {64, uint64_t(d.Hs), nl, uint64_t(capacity)};
-  const uint64_t strides[3] = {128, uint64_t(d.Hs) * 128, nl * uint64_t(d.Hs) * 128};
-  const uint32_t box[4] = {64, 1, 8, 1};
-  e = make_tmap_bf16(&tv, values, 4, dims, strides, box, 128);
+  const uint64_t lpg = uint64_t(d.B) / 4;  // lines of one 16-key group
+  const uint64_t dims[5] = {64, uint64_t(d.Hs), lpg, nl / lpg, uint64_t(capacity)};
+  const uint64_t strides[4] = {128, uint64_t(d.Hs) * 128, lpg * uint64_t(d.Hs) * 128,
+                               nl * uint64_t(d.Hs) * 128};
+  const uint32_t box[5] = {64, 1, 8, 4, 1};
+  e = make_tmap_bf16(&tv, values, 5, dims, strides, box, 128);
   if (e != cudaSuccess) return e;
   qk::Params p{};
   p.cu_seqlens = d.cu_seqlens;

@@ -142,7 +142,7 @@ def sender_qk(lengths, Hs: int, d: int, dtype: str, rng: np.random.Generator,
     for L in lengths:
         q = rng.standard_normal((L, Hs, d), dtype=np.float32) * np.float32(qk_gain)
         k = rng.standard_normal((L, Hs, d), dtype=np.float32) * np.float32(qk_gain)
-        if sink_gain != 0.0:
+        if sink_gain != 0.0 and L > 0:  # an empty sequence has no sink
             u = q.mean(axis=0, dtype=np.float32)                      # [Hs, d]
             u = u / np.linalg.norm(u, axis=1, keepdims=True).astype(np.float32)
             ns = min(SINK_TOKENS, L)

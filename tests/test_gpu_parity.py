@@ -124,6 +124,24 @@ def test_large_workload_sampled():
     assert torch.isfinite(O.float()).all()
 
 
+def test_long_b64_sequence_past_256_key_blocks():
+    """One 16,500-token sequence at B = 64 (258 key blocks): the statistics
+    take the scalar two-pass kernel (the tensor-core one keeps per-block
+    partials for at most 256 key blocks in TMEM) while extraction and the
+    fused kernel stay on the tensor cores, with block-map entries past 256.
+    Sampled query blocks, the last ones included, against the oracle."""
+    w, x = synth.small_case([16500], 8, 16, 4, 128, 64, 0.95)
+    ctx = _ctx_of(w)
+    assert mfb.path_info(ctx, w.Hr, w.Hkv) == {"stats_tc": False, "extract_tc": True,
+                                                "mapped_av_tc": True}
+    gpu = par.run_gpu(ctx, x.Q.cuda(), x.K.cuda(), x.V.cuda(), x.W.cuda(), w.Hkv, w.tau)
+    picks = [(0, 0), (0, 1), (0, 128), (0, 255), (0, 256), (0, 257)]
+    n, ex, worst = par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, gpu,
+                                            picks, torch.bfloat16, label="long B = 64")
+    assert n == len(picks) and ex <= 1
+    assert torch.isfinite(gpu[3].float()).all()
+
+
 def test_multi_receiver_workload_as_specified():
     """One sender state of 8 layers, each compressed once, serves receiver r1
     (6 layers) and receiver r2 (4 layers) through the layer table; every

@@ -191,13 +191,18 @@ mf_status mf_block_stats(const mf_attn_desc* desc, const void* Q, const void* K,
   return mf_block_stats_range(desc, Q, K, lse, mass, 0, sz.nqb, ws, ws_bytes, stream);
 }
 
+// A NULL pointer is accepted for a buffer that is empty at the sizes given.
+static bool present(const void* p, int64_t elements) { return p != nullptr || elements == 0; }
+
 mf_status mf_block_stats_range(const mf_attn_desc* desc, const void* Q, const void* K,
                                float* lse, float* mass, int64_t qb_begin, int64_t qb_end,
                                void* ws, size_t ws_bytes, mf_stream_t stream) {
   Sizes sz;
   mf_status st = check_desc(desc, &sz);
   if (st != MF_OK) return st;
-  if (!Q || !K || !lse || !mass) return fail(MF_ERR_INVALID_ARG, "Q, K, lse or mass is NULL");
+  if (!present(Q, sz.ntok) || !present(K, sz.ntok) || !present(lse, sz.ntok) ||
+      !present(mass, sz.nblocks))
+    return fail(MF_ERR_INVALID_ARG, "Q, K, lse or mass is NULL");
   st = check_range(sz, qb_begin, qb_end);
   if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
@@ -231,7 +236,8 @@ size_t mf_select_extract_workspace(const mf_attn_desc* desc) {
 
 static mf_status check_cache(const mf_csr_cache* c, const mf_attn_desc& d, const Sizes& sz) {
   if (!c) return fail(MF_ERR_INVALID_ARG, "cache is NULL");
-  if (!c->row_ptr || !c->col_idx || !c->qb_seq || !c->qb_idx || !c->values)
+  if (!c->row_ptr || !present(c->col_idx, c->nnz_capacity) || !present(c->qb_seq, sz.nqb) ||
+      !present(c->qb_idx, sz.nqb) || !present(c->values, c->nnz_capacity))
     return fail(MF_ERR_INVALID_ARG, "cache has a NULL array");
   if (c->Hs != d.Hs || c->B != d.B || c->dt != d.dt)
     return fail(MF_ERR_INVALID_ARG, "cache Hs/B/dtype differ from the descriptor");
@@ -259,7 +265,9 @@ mf_status mf_select_extract_range(const mf_attn_desc* desc, const void* Q, const
   mf_status st = check_desc(desc, &sz);
   if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
-  if (!Q || !K || !lse || !mass) return fail(MF_ERR_INVALID_ARG, "Q, K, lse or mass is NULL");
+  if (!present(Q, sz.ntok) || !present(K, sz.ntok) || !present(lse, sz.ntok) ||
+      !present(mass, sz.nblocks))
+    return fail(MF_ERR_INVALID_ARG, "Q, K, lse or mass is NULL");
   if (!(tau > 0.0) || !std::isfinite(tau)) return fail(MF_ERR_INVALID_ARG, "tau must be > 0");
   st = check_cache(out, d, sz);
   if (st != MF_OK) return st;
@@ -353,7 +361,7 @@ static mf_status check_av(const mf_csr_cache* cache, const mf_attn_desc* desc, i
   const mf_attn_desc& d = *desc;
   st = check_cache(cache, d, *sz);
   if (st != MF_OK) return st;
-  if (!v || !v->V) return fail(MF_ERR_INVALID_ARG, "V is NULL");
+  if (!v || !present(v->V, sz->ntok)) return fail(MF_ERR_INVALID_ARG, "V is NULL");
   if (v->d != d.d) return fail(MF_ERR_INVALID_ARG, "V head dim differs from the descriptor");
   if (v->Hkv < 1 || Hr < 1 || Hr % v->Hkv != 0)
     return fail(MF_ERR_INVALID_ARG, "Hr must be a positive multiple of Hkv");
@@ -398,7 +406,7 @@ mf_status mf_mapped_av_range(const mf_csr_cache* cache, const mf_attn_desc* desc
   mf_status st = check_av(cache, desc, Hr, v, &sz);
   if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
-  if (!W || !O) return fail(MF_ERR_INVALID_ARG, "W or O is NULL");
+  if (!W || !present(O, sz.ntok)) return fail(MF_ERR_INVALID_ARG, "W or O is NULL");
   st = check_range(sz, qb_begin, qb_end);
   if (st != MF_OK) return st;
   const bool tc = mapped_av_tc_supported(d, Hr, *v);
@@ -474,7 +482,8 @@ mf_status mf_extract(const mf_attn_desc* desc, const void* Q, const void* K, con
   mf_status st = check_desc(desc, &sz);
   if (st != MF_OK) return st;
   const mf_attn_desc& d = *desc;
-  if (!Q || !K || !lse) return fail(MF_ERR_INVALID_ARG, "Q, K or lse is NULL");
+  if (!present(Q, sz.ntok) || !present(K, sz.ntok) || !present(lse, sz.ntok))
+    return fail(MF_ERR_INVALID_ARG, "Q, K or lse is NULL");
   st = check_cache(cache, d, sz);
   if (st != MF_OK) return st;
   if (!ws || !aligned256(ws) || ws_bytes < extract_ws(d, sz, nullptr, nullptr, nullptr))

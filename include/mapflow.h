@@ -24,6 +24,10 @@
  *    device (a bounded wait that gave up, a CSR capacity overflow) set a
  *    per-device status word that mf_sync_status() reads and clears.
  *  - The text of the last error of the calling thread: mf_last_error().
+ *  - A buffer that is empty at the descriptor's sizes may be NULL: Q, K, lse,
+ *    V and O when ntok = 0; mass when there are no causal blocks; a cache's
+ *    col_idx and values when nnz_capacity = 0, its qb_seq and qb_idx when
+ *    nqb_total = 0.  Every other NULL pointer is MF_ERR_INVALID_ARG.
  *
  * Notation: ntok packed tokens over nseq sequences (cu_seqlens prefix sums);
  * Hs sender heads; Hr receiver heads; Hkv receiver KV heads; d head dim;

@@ -59,6 +59,34 @@ def _desc(Hs=4, d=64, B=64, cu=(0, 512), dt=mfb.MF_F32):
     return dsc, host
 
 
+def test_null_is_accepted_only_for_empty_buffers(lib):
+    """Empty buffers may be NULL (a batch without tokens): the calls then get
+    past the argument checks (here, with no GPU, to MF_ERR_CUDA); the same
+    NULL with tokens present is MF_ERR_INVALID_ARG."""
+    P = C.c_void_p
+    empty, _h0 = _desc(cu=(0, 0, 0))
+    full, _h1 = _desc(cu=(0, 100))
+    ws = P(256)
+    need = lib.mf_block_stats_workspace(C.byref(empty))
+    assert lib.mf_block_stats(C.byref(empty), None, None, None, None, ws, need, None) == \
+        mfb.MF_ERR_CUDA
+    assert lib.mf_block_stats(C.byref(full), None, None, None, None, ws, 1 << 20, None) == \
+        mfb.MF_ERR_INVALID_ARG
+    # no query blocks: only row_ptr must exist
+    cache0 = mfb.CsrCache(0, 0, 16, None, None, None, None, 4, 64, mfb.MF_F32, 2, 0x1000)
+    need = lib.mf_select_extract_workspace(C.byref(empty))
+    assert lib.mf_select_extract(C.byref(empty), None, None, None, None, 0.9,
+                                 C.byref(cache0), ws, need, None) == mfb.MF_ERR_CUDA
+    cache1 = mfb.CsrCache(2, 0, 16, None, None, None, None, 4, 64, mfb.MF_F32, 1, 0x1000)
+    assert lib.mf_select_extract(C.byref(full), P(16), P(16), P(16), P(16), 0.9,
+                                 C.byref(cache1), ws, 1 << 20, None) == mfb.MF_ERR_INVALID_ARG
+    v0 = mfb.VDesc(None, None, 16, 0, 0, 2, 64)
+    assert lib.mf_mapped_av(C.byref(cache0), C.byref(empty), 4, P(16), C.byref(v0), None,
+                            ws, 1 << 20, None) == mfb.MF_ERR_CUDA
+    assert lib.mf_mapped_av(C.byref(cache0), C.byref(empty), 4, None, C.byref(v0), None,
+                            ws, 1 << 20, None) == mfb.MF_ERR_INVALID_ARG  # W is never empty
+
+
 def test_argument_errors_return_before_any_launch(lib):
     dsc, host = _desc()
     P = C.c_void_p

@@ -41,14 +41,28 @@ def _small(lengths, Hs, Hr, Hkv, d, B, tau, dtype="bf16", band_bias=2.0, band_wi
     # last head group (8 + 4); the fused step runs the scalar kernel
     dict(lengths=[700, 257], Hs=12, Hr=8, Hkv=4, d=128, B=128, tau=0.95),
     dict(lengths=[450, 1], Hs=12, Hr=8, Hkv=4, d=128, B=64, tau=0.9),
+    # empty sequences between non-empty ones, all three stages on the tensor cores
+    dict(lengths=[0, 300, 0, 129], Hs=8, Hr=16, Hkv=4, d=128, B=64, tau=0.9),
 ], ids=["bf16_b64_varlen", "bf16_b128_hs40", "bf16_b64_hs32", "bf16_d64",
-        "f32_d128_b128", "f32_empty_seq", "bf16_b128_hs12", "bf16_b64_hs12"])
+        "f32_d128_b128", "f32_empty_seq", "bf16_b128_hs12", "bf16_b64_hs12",
+        "bf16_empty_seqs_tc"])
 def test_small_cases_every_block(case):
     w, x, ctx, gpu = _small(**case)
     dt = w.torch_dtype
     n, ex, worst = par.compare_query_blocks(ctx, x.Q, x.K, x.V, x.W, w.Hkv, w.tau, gpu,
                                             par.all_picks(ctx), dt, label="small cases")
     assert ex <= max(1, n // 50)
+
+
+def test_batch_without_tokens():
+    """Every sequence empty: the three calls launch nothing, report no error
+    and return an empty cache and an empty O."""
+    w, x = synth.small_case([0, 0], 8, 16, 4, 128, 64, 0.9)
+    ctx = _ctx_of(w)
+    lse, mass, cache, O = par.run_gpu(ctx, x.Q.cuda(), x.K.cuda(), x.V.cuda(), x.W.cuda(),
+                                      w.Hkv, w.tau)
+    mfb.sync_status()
+    assert cache.nnz == 0 and O.shape[0] == 0 and lse.numel() == 0
 
 
 def test_tiny_f32_workload_every_block():

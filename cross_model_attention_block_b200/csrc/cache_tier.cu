@@ -26,9 +26,13 @@ size_t elem_bytes(mf_dtype dt) { return dt == MF_F32 ? 4 : 2; }
 
 mf_status same_layout(const mf_csr_cache* a, const mf_csr_cache* b) {
   if (!a || !b) return fail(MF_ERR_INVALID_ARG, "cache is NULL");
-  if (!a->row_ptr || !a->col_idx || !a->qb_seq || !a->qb_idx || !a->values || !b->row_ptr ||
-      !b->col_idx || !b->qb_seq || !b->qb_idx || !b->values)
-    return fail(MF_ERR_INVALID_ARG, "cache has a NULL array");
+  // an array may be NULL only where it is empty (no entries, no query blocks)
+  for (const mf_csr_cache* c : {a, b}) {
+    const bool rows = c->nqb_total == 0, entries = c->nnz_capacity == 0;
+    if (!c->row_ptr || (!c->qb_seq && !rows) || (!c->qb_idx && !rows) ||
+        (!c->col_idx && !entries) || (!c->values && !entries))
+      return fail(MF_ERR_INVALID_ARG, "cache has a NULL array");
+  }
   if (a->nqb_total != b->nqb_total || a->Hs != b->Hs || a->B != b->B || a->dt != b->dt)
     return fail(MF_ERR_INVALID_ARG, "caches differ in nqb_total, Hs, B or dtype");
   if (a->nqb_total < 0 || a->nnz_capacity < 0 || b->nnz_capacity < 0 || a->Hs < 1 ||

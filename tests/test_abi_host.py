@@ -334,6 +334,15 @@ def test_cache_tier_checks_layouts_and_ranges(lib):
     with pytest.raises(mfb.MapflowError) as e:
         mfb.cache_fetch(a, mfb.Cache(ctx, device="cpu"), (2, 99))
     assert "range" in str(e.value)
+    # arrays may be NULL only where they are empty
+    rp = np.zeros(1, np.int64)
+    none = mfb.CsrCache(0, 0, rp.ctypes.data, None, None, None, None, 8, 64, mfb.MF_BF16, 1,
+                        0x1000)
+    assert lib.mf_cache_fetch(C.byref(none), C.byref(none), 0, 0, None) == mfb.MF_OK
+    holes = mfb.CsrCache(0, 4, rp.ctypes.data, None, None, None, None, 8, 64, mfb.MF_BF16, 1,
+                         0x1000)
+    assert lib.mf_cache_fetch(C.byref(holes), C.byref(holes), 0, 0, None) == \
+        mfb.MF_ERR_INVALID_ARG
 
 
 def test_overlap_chunk_ranges_cover_the_rows():
